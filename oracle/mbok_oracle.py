@@ -1,0 +1,233 @@
+"""CPU oracle for the multi-Boolean-kernel (MBOK) linear layer.
+
+TEST INFRASTRUCTURE.  Only the tests, the smoke check of the package entry
+point and the CPU-baseline leg of the benchmark may import or run this module.
+The product (the C ABI and its Python binding) never calls it, and it shares
+no code with the CUDA path: it reads only the layout definition restated
+below and the seeded inputs.
+
+What it computes, and where the method defines it
+-------------------------------------------------
+Source pages: "Highly Efficient and Effective LLMs with Multi-Boolean
+Architectures" (ICLR 2026; arXiv 2505.22811) as summarised by the Paper-Notes
+page (section "方法详解 / 关键设计") and by the gist.science technical summaries
+(Italian 2A-2D, Dutch "Methodologie", Spanish 2A-2D).
+
+* Representation (Paper-Notes, 关键设计, "多核布尔参数表示"): a weight matrix
+  is approximated by a weighted sum of K Boolean matrices,
+  W ~= sum_k alpha_k * B_k with B_k in {-1,+1}^{M x N}.
+* Grouping (Paper-Notes, 关键设计, "分组量化策略"; ablation table: group
+  size 128 is the usual choice): every 128-column group of a row has its own
+  scale, so alpha_{k,r,g} multiplies B_k[r, 128g:128g+128].
+* The linear op (Paper-Notes, 关键设计: "Wx decomposes into K Boolean
+  matrix-vector products"): y = W x with that W.  The oracle reconstructs W in
+  fp64 (exact: each entry is a sum of at most four fp16 values times +-1) and
+  multiplies with a float64 BLAS product.
+* Scale for a fixed sign matrix (Paper-Notes, 关键设计, "缩放因子的高效优化":
+  closed-form least squares): for B = sign(R) the least-squares scale of a
+  group is mean|R| over the group.
+* Kernel k fits what kernels 1..k-1 left (Dutch technical summary,
+  "Successive SVID"; Spanish 2B "Extracción Sucesiva": each later kernel
+  approximates the residual of the previous approximation; Paper-Notes,
+  训练策略: greedy initialisation).  Here: R_0 = W, B_k = sign(R_{k-1}),
+  alpha_k = mean|R_{k-1}| per (row, group), R_k = R_{k-1} - alpha_k B_k.
+
+Readings where the pages are silent (each one is listed in the design notes):
+  sign(0) = +1 (and -0.0 >= 0 so also +1); packer input 0 also maps to +1;
+  a stored bit 1 means +1;
+  the greedy residual keeps R in fp32, sums |R| over a group in fp64 in column
+  order j = 0..127, divides by 128 (exact), rounds once from fp64 to fp16
+  (nearest, ties to even), and updates R <- R - alpha_hat * b with the fp16
+  value, as one fp32 subtraction;
+  N must be a multiple of 128 (no ragged group).
+
+Bit layout "V1" (the pages give none; this is the library's storage format):
+  rows are cut into tiles of 128 (the last tile is padded; pad rows are
+  ignored), columns into groups of 128, each group into four 32-column chunks.
+  The packed array is a flat uint32 array ordered
+      [row tile rt][group g][row in tile r_in][chunk c][kernel k]
+  and bit i (least significant = 0) of a word holds column 128 g + 32 c + i.
+  So one row's record for one group is 4*K consecutive words, and for one
+  32-column chunk the K kernels' words sit side by side.
+Scales alpha are fp16 stored [M][N/128][K] (kernel index fastest).
+
+Parity pins: see tests/test_oracle_pins.py (brute force in exact rational
+arithmetic, flip invariance, level count, least-squares closed form, residual
+norm identity, the XNOR/popcount identity, a hand-worked layout example, the
+dense special case and a rounding case for the fp64->fp16 step).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+GROUP = 128        # columns per scale group
+TILE_ROWS = 128    # rows per layout tile
+CHUNKS = GROUP // 32
+
+
+# --------------------------------------------------------------------------
+# Layout sizes and addressing (restated from the V1 definition above)
+# --------------------------------------------------------------------------
+
+def n_groups(N: int) -> int:
+    if N % GROUP:
+        raise ValueError("N must be a multiple of 128")
+    return N // GROUP
+
+
+def n_row_tiles(M: int) -> int:
+    return (M + TILE_ROWS - 1) // TILE_ROWS
+
+
+def packed_words(K: int, M: int, N: int) -> int:
+    return n_row_tiles(M) * n_groups(N) * TILE_ROWS * CHUNKS * K
+
+
+def alpha_elems(K: int, M: int, N: int) -> int:
+    return M * n_groups(N) * K
+
+
+def word_and_bit(K: int, M: int, N: int, k: int, r: int, j: int) -> tuple[int, int]:
+    """Word index and bit position that hold kernel k, row r, column j."""
+    G = n_groups(N)
+    rt, r_in = divmod(r, TILE_ROWS)
+    g, jj = divmod(j, GROUP)
+    c, bit = divmod(jj, 32)
+    word = ((rt * G + g) * TILE_ROWS + r_in) * (CHUNKS * K) + c * K + k
+    return word, bit
+
+
+# --------------------------------------------------------------------------
+# Packing and unpacking
+# --------------------------------------------------------------------------
+
+def pack_signs(signs: np.ndarray) -> np.ndarray:
+    """int8 signs [K][M][N] -> V1 words.  An entry >= 0 is stored as bit 1 (+1)."""
+    K, M, N = signs.shape
+    G, RT = n_groups(N), n_row_tiles(M)
+    bits = np.zeros((K, RT * TILE_ROWS, N), dtype=np.uint64)
+    bits[:, :M, :] = signs >= 0
+    b = bits.reshape(K, RT, TILE_ROWS, G, CHUNKS, 32)
+    words = np.zeros((K, RT, TILE_ROWS, G, CHUNKS), dtype=np.uint64)
+    for i in range(32):
+        words |= b[..., i] << np.uint64(i)
+    # storage order [rt][g][r_in][c][k]
+    return np.ascontiguousarray(words.transpose(1, 3, 2, 4, 0)).astype(np.uint32).ravel()
+
+
+def unpack_rows(packed: np.ndarray, K: int, M: int, N: int, rows) -> np.ndarray:
+    """V1 words -> b in {-1,+1}, int8 [K][len(rows)][N], for the listed rows."""
+    G, RT = n_groups(N), n_row_tiles(M)
+    rows = np.asarray(rows, dtype=np.int64)
+    w = np.asarray(packed, dtype=np.uint32).reshape(RT, G, TILE_ROWS, CHUNKS, K)
+    sel = w[rows // TILE_ROWS, :, rows % TILE_ROWS, :, :]          # [R][G][C][K]
+    shifts = np.arange(32, dtype=np.uint32)
+    bits = (sel[..., None] >> shifts) & np.uint32(1)                 # [R][G][C][K][32]
+    bits = bits.transpose(3, 0, 1, 2, 4).reshape(K, len(rows), N)   # [K][R][N]
+    return np.where(bits == 1, 1, -1).astype(np.int8)
+
+
+def unpack_bits(packed: np.ndarray, K: int, M: int, N: int) -> np.ndarray:
+    return unpack_rows(packed, K, M, N, np.arange(M))
+
+
+# --------------------------------------------------------------------------
+# The weight and the linear op
+# --------------------------------------------------------------------------
+
+def reconstruct_rows(packed, alpha, K: int, M: int, N: int, rows) -> np.ndarray:
+    """fp64 W[rows, :] with W_rj = sum_k alpha_{k,r,floor(j/128)} * b_{k,r,j}."""
+    G = n_groups(N)
+    rows = np.asarray(rows, dtype=np.int64)
+    b = unpack_rows(packed, K, M, N, rows).astype(np.float64)        # [K][R][N]
+    a = np.asarray(alpha, dtype=np.float16).reshape(M, G, K)[rows].astype(np.float64)  # [R][G][K]
+    a_cols = np.repeat(a, GROUP, axis=1)                             # [R][N][K]
+    W = np.zeros((len(rows), N), dtype=np.float64)
+    for k in range(K):
+        W += a_cols[:, :, k] * b[k]
+    return W
+
+
+def reconstruct_W(packed, alpha, K: int, M: int, N: int) -> np.ndarray:
+    return reconstruct_rows(packed, alpha, K, M, N, np.arange(M))
+
+
+def as_f64(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Activations to fp64 (exact for fp32 and bf16)."""
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    if dtype == "bf16":
+        return (np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def linear(packed, alpha, K: int, M: int, N: int, x, x_dtype: str, rows=None):
+    """y[b][r] = sum_j W_rj x[b][j] and E[b][r] = sum_j |W_rj x[b][j]| in fp64.
+
+    x is [batch][N] (fp32, or bf16 bit patterns).  rows selects output rows
+    (default all).  E feeds the per-element tolerance |y - y_ref| <= 1e-3 E + 1e-6.
+    """
+    rows = np.arange(M) if rows is None else np.asarray(rows, dtype=np.int64)
+    W = reconstruct_rows(packed, alpha, K, M, N, rows)
+    xf = as_f64(x, x_dtype).reshape(-1, N)
+    y = xf @ W.T
+    E = np.abs(xf) @ np.abs(W).T
+    return y, E
+
+
+# --------------------------------------------------------------------------
+# Greedy residual binarisation
+# --------------------------------------------------------------------------
+
+def residual_binarize(W: np.ndarray, K: int):
+    """fp32 W [M][N] -> (signs int8 [K][M][N], alpha fp16 [M][G][K], R_K fp32 [M][N]).
+
+    For k = 1..K, per (row r, group g):
+      b     = sign(R_{k-1}), sign(0) = +1
+      alpha = RN_fp16( (sum_{j=0..127} |R_{k-1}|, fp64, in column order) / 128 )
+      R_k   = R_{k-1} - alpha * b     (fp32, alpha the fp16 value, one rounding)
+    """
+    W = np.asarray(W, dtype=np.float32)
+    M, N = W.shape
+    G = n_groups(N)
+    R = W.copy()
+    signs = np.empty((K, M, N), dtype=np.int8)
+    alpha = np.empty((M, G, K), dtype=np.float16)
+    for k in range(K):
+        b = np.where(R >= np.float32(0), np.int8(1), np.int8(-1))
+        A = np.abs(R).astype(np.float64).reshape(M, G, GROUP)
+        acc = np.zeros((M, G), dtype=np.float64)
+        for j in range(GROUP):          # the prescribed summation order
+            acc = acc + A[:, :, j]
+        a16 = (acc / 128.0).astype(np.float16)
+        a32 = np.repeat(a16.astype(np.float32), GROUP, axis=1)      # [M][N]
+        R = (R - a32 * b.astype(np.float32)).astype(np.float32)
+        signs[k] = b
+        alpha[:, :, k] = a16
+    return signs, alpha, R
+
+
+# --------------------------------------------------------------------------
+# Tolerance
+# --------------------------------------------------------------------------
+
+def within_tolerance(y, y_ref, E, rel: float = 1e-3, abs_: float = 1e-6) -> np.ndarray:
+    """Per-element bound |y - y_ref| <= rel * E + abs_ (boolean mask)."""
+    y = np.asarray(y, dtype=np.float64)
+    return np.abs(y - y_ref) <= rel * E + abs_
+
+
+def rel_l2(y, y_ref) -> float:
+    y = np.asarray(y, dtype=np.float64)
+    den = float(np.linalg.norm(y_ref))
+    return float(np.linalg.norm(y - y_ref)) / (den if den > 0 else 1.0)
+
+
+def levels(K: int, alphas) -> set:
+    """The set {sum_k s_k alpha_k : s in {-1,+1}^K} (at most 2^K weight levels)."""
+    out = set()
+    for m in range(1 << K):
+        out.add(math.fsum((1.0 if (m >> k) & 1 else -1.0) * float(alphas[k]) for k in range(K)))
+    return out

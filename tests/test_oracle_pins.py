@@ -1,0 +1,280 @@
+"""Pins for the CPU oracle, each against something other than the oracle itself.
+
+Every check cites the fact it rests on.  A plausible slip in the oracle (a
+dropped kernel, a wrong sign, a transposed index, a wrong word or bit order, a
+double rounding of the scale) fails at least one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import mbok_oracle as O
+from boolean_weight_matmul_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _signs_alpha_x(K, M, N, seed, x_dtype="f32"):
+    s = wl.random_signs(K, M, N, seed)
+    a = wl.alpha_abs_normal(K, M, N, seed + 1)
+    x = wl.x_normal(1, N, seed + 2, x_dtype)
+    return s, a, x
+
+
+# --------------------------------------------------------------------------
+# Layout (O6): hand-worked words, scalar addressing, round trip
+# --------------------------------------------------------------------------
+
+def test_layout_hand_worked_example():
+    # tests/golden/layout_k2_1x128.txt: words derived by hand from the layout rules.
+    with open(os.path.join(GOLDEN, "layout_k2_1x128.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    assert lines[0] == "K=2 M=1 N=128"
+    expect = [int(t, 16) for t in lines[1].split()]
+    j = np.arange(128)
+    signs = np.stack([np.where(j % 3 == 0, 1, -1), np.where(j < 40, 1, -1)]).astype(np.int8)[:, None, :]
+    packed = O.pack_signs(signs)
+    assert packed.shape == (O.packed_words(2, 1, 128),) == (1024,)
+    assert [int(v) for v in packed[:8]] == expect
+    assert not packed[8:].any()
+
+
+def test_layout_scalar_addressing_ragged():
+    # Vectorised packer agrees bit by bit with the scalar address rule, with a
+    # ragged last row tile (M=130) and three groups.
+    K, M, N = 3, 130, 384
+    s = wl.random_signs(K, M, N, 11, p_zero=0.05)
+    packed = O.pack_signs(s)
+    r = np.random.default_rng(5)
+    for _ in range(3000):
+        k, row, col = int(r.integers(K)), int(r.integers(M)), int(r.integers(N))
+        w, b = O.word_and_bit(K, M, N, k, row, col)
+        assert (int(packed[w]) >> b) & 1 == int(s[k, row, col] >= 0)
+
+
+def test_layout_round_trip_and_zero_maps_to_plus_one():
+    K, M, N = 4, 129, 256
+    s = wl.random_signs(K, M, N, 12, p_zero=0.1)
+    b = O.unpack_bits(O.pack_signs(s), K, M, N)
+    assert np.array_equal(b, np.where(s >= 0, 1, -1))
+
+
+# --------------------------------------------------------------------------
+# The linear op (O1 brute force, O2 flips, O3 levels, O5 XNOR, O7 dense)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K", [1, 2, 3])
+def test_brute_force_exact_rational(K):
+    # y_r = sum_j (sum_k alpha_{k,r,g(j)} s_{k,r,j}) x_j in exact rational
+    # arithmetic, straight from the int8 signs (Paper-Notes 关键设计:
+    # W ~= sum_k alpha_k B_k with group-wise scales).
+    M, N = 3, 256
+    s, a, x = _signs_alpha_x(K, M, N, 100 + K)
+    y, E = O.linear(O.pack_signs(s), a, K, M, N, x, "f32")
+    xf = [Fraction(float(v)) for v in x[0]]
+    for r in range(M):
+        acc = Fraction(0)
+        for j in range(N):
+            w = sum(Fraction(float(a[r, j // 128, k])) * int(s[k, r, j] >= 0 and 1 or -1) for k in range(K))
+            acc += w * xf[j]
+        assert abs(y[0, r] - float(acc)) <= 1e-14 * E[0, r] + 1e-300
+
+
+def test_per_kernel_decomposition_agrees():
+    # The pages' form "Wx = K Boolean mat-vecs" (Paper-Notes 关键设计):
+    # sum_k alpha_k (B_k x), evaluated kernel by kernel and group by group.
+    K, M, N = 3, 5, 384
+    s, a, x = _signs_alpha_x(K, M, N, 7)
+    y, E = O.linear(O.pack_signs(s), a, K, M, N, x, "f32")
+    xf = x[0].astype(np.float64)
+    y2 = np.zeros(M)
+    for k in range(K):
+        for g in range(N // 128):
+            sl = slice(128 * g, 128 * g + 128)
+            y2 += a[:, g, k].astype(np.float64) * (s[k][:, sl].astype(np.float64) @ xf[sl])
+    assert np.all(np.abs(y[0] - y2) <= 1e-13 * E[0])
+
+
+def test_flip_invariance_bitwise():
+    # Negating alpha_k and flipping every sign of B_k leaves W, hence y,
+    # unchanged exactly (IEEE negation is exact).
+    K, M, N = 3, 7, 256
+    s, a, x = _signs_alpha_x(K, M, N, 21)
+    y0, _ = O.linear(O.pack_signs(s), a, K, M, N, x, "f32")
+    for k in range(K):
+        s2, a2 = s.copy(), a.copy()
+        s2[k] = -s2[k]
+        a2[:, :, k] = -a2[:, :, k]
+        y1, _ = O.linear(O.pack_signs(s2), a2, K, M, N, x, "f32")
+        assert np.array_equal(y0, y1)
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+def test_at_most_2_pow_K_levels(K):
+    # Paper-Notes 关键设计: K kernels give 2^K weight levels.
+    M, N = 4, 256
+    s = wl.random_signs(K, M, N, 30 + K)
+    a = wl.alpha_decaying(K, M, N, 40 + K)
+    W = O.reconstruct_W(O.pack_signs(s), a, K, M, N)
+    for r in range(M):
+        for g in range(N // 128):
+            vals = set(W[r, 128 * g:128 * g + 128].tolist())
+            lev = O.levels(K, a[r, g, :])
+            assert vals <= lev
+            assert len(vals) <= 2 ** K
+            if K <= 3:  # 128 random columns hit all 2^K sign patterns
+                assert vals == lev
+
+
+def test_xnor_popcount_identity():
+    # K=1, alpha=1, x in {-1,+1}^N: b.x = 2*popcount(XNOR(b, x)) - N
+    # (the XNOR+popcount form named on the Paper-Notes page, 关键设计).
+    M, N = 6, 512
+    s = wl.random_signs(1, M, N, 50)
+    a = np.ones((M, N // 128, 1), dtype=np.float16)
+    xs = np.where(np.random.default_rng(51).random(N) < 0.5, -1.0, 1.0).astype(np.float32)
+    y, _ = O.linear(O.pack_signs(s), a, 1, M, N, xs[None, :], "f32")
+    xbits = sum(1 << j for j in range(N) if xs[j] > 0)
+    for r in range(M):
+        bbits = sum(1 << j for j in range(N) if s[0, r, j] >= 0)
+        xnor = ~(bbits ^ xbits) & ((1 << N) - 1)
+        assert y[0, r] == 2 * bin(xnor).count("1") - N
+
+
+def test_dense_special_case():
+    # K=1 with one scale a for every group: y = a * (B x), B x by a naive loop.
+    M, N = 4, 256
+    s = wl.random_signs(1, M, N, 60)
+    aval = np.float16(0.037)
+    a = np.full((M, N // 128, 1), aval, dtype=np.float16)
+    x = wl.x_normal(1, N, 61, "f32")
+    y, E = O.linear(O.pack_signs(s), a, 1, M, N, x, "f32")
+    for r in range(M):
+        acc = 0.0
+        for j in range(N):
+            acc += (1.0 if s[0, r, j] >= 0 else -1.0) * float(x[0, j])
+        assert abs(y[0, r] - float(aval) * acc) <= 1e-12 * E[0, r]
+
+
+def test_bf16_activations_exact_widening():
+    # bf16 bit pattern 0x3FC0 is 1.5, 0xC020 is -2.5; fp64 widening is exact.
+    x = np.array([[0x3FC0, 0xC020]], dtype=np.uint16)
+    assert O.as_f64(x, "bf16").tolist() == [[1.5, -2.5]]
+
+
+# --------------------------------------------------------------------------
+# Residual binarisation (O4)
+# --------------------------------------------------------------------------
+
+def test_residual_k1_closed_form_least_squares():
+    # Paper-Notes 关键设计 (closed-form least squares for alpha given B):
+    # for B = sign(W) the optimum is a* = mean|W| over the group; the stored
+    # fp16 scale is the fp16 value nearest to it, so it beats both fp16 neighbours.
+    M, N = 8, 256
+    W = wl.w_normal(M, N, 70)
+    s, a, R = O.residual_binarize(W, 1)
+    assert np.array_equal(s[0], np.where(W >= 0, 1, -1))
+    for r in range(M):
+        for g in range(N // 128):
+            w = W[r, 128 * g:128 * g + 128].astype(np.float64)
+            exact_mean = math.fsum(abs(v) for v in w) / 128.0
+            assert a[r, g, 0] == np.float16(exact_mean)
+            b = np.where(w >= 0, 1.0, -1.0)
+
+            def f(al):
+                return float(np.sum((w - al * b) ** 2))
+            h = a[r, g, 0]
+            up = np.nextafter(h, np.float16(np.inf))
+            dn = np.nextafter(h, np.float16(-np.inf))
+            assert f(float(h)) <= f(float(up)) and f(float(h)) <= f(float(dn))
+
+
+def test_sign_and_scale_jointly_optimal_brute_force():
+    # On an 8-entry toy group, over all 2^8 sign vectors with their optimal
+    # scale <w,b>/8, the best fit is b = sign(w) with scale mean|w|.
+    r = np.random.default_rng(71)
+    for _ in range(20):
+        w = r.standard_normal(8)
+        best = None
+        for m in range(256):
+            b = np.array([1.0 if (m >> i) & 1 else -1.0 for i in range(8)])
+            al = float(w @ b) / 8.0
+            err = float(np.sum((w - al * b) ** 2))
+            if best is None or err < best[0] - 1e-15:
+                best = (err, b, al)
+        assert np.array_equal(best[1], np.where(w >= 0, 1.0, -1.0)) or np.array_equal(best[1], -np.where(w >= 0, 1.0, -1.0))
+        assert abs(abs(best[2]) - float(np.mean(np.abs(w)))) < 1e-12
+
+
+def test_residual_norm_identity_and_monotone():
+    # Each kernel fits the residual of the previous ones (Dutch technical
+    # summary, Successive SVID; Spanish 2B).  Per group, with S = sum|R_{k-1}|:
+    #   ||R_k||^2 = ||R_{k-1}||^2 - 2 alpha S + 128 alpha^2   (exact algebra; the
+    # fp32 rounding of R_k is the only slack), and ||R_k|| never grows.
+    K, M, N = 3, 16, 512
+    W = wl.w_normal(M, N, 72)
+    s, a, RK = O.residual_binarize(W, K)
+    R = W.astype(np.float64)
+    prev = None
+    for k in range(K):
+        for r in range(M):
+            for g in range(N // 128):
+                seg = R[r, 128 * g:128 * g + 128]
+                S = float(np.sum(np.abs(seg)))
+                al = float(a[r, g, k])
+                b = s[k, r, 128 * g:128 * g + 128].astype(np.float64)
+                assert np.array_equal(b, np.where(seg >= 0, 1.0, -1.0))
+                assert a[r, g, k] == np.float16(S / 128.0)
+                new = seg - al * b
+                pred = float(np.sum(seg ** 2)) - 2 * al * S + 128 * al * al
+                assert abs(float(np.sum(new ** 2)) - pred) <= 1e-12 * max(1.0, float(np.sum(seg ** 2)))
+        R = (R.astype(np.float32) - np.repeat(a[:, :, k].astype(np.float32), 128, axis=1) * s[k].astype(np.float32)).astype(np.float64)
+        nrm = float(np.linalg.norm(R))
+        assert prev is None or nrm <= prev
+        prev = nrm
+    assert np.array_equal(R.astype(np.float32), RK)
+    # the kernels reconstruct W up to the final residual (fp32 steps only)
+    Wk = O.reconstruct_W(O.pack_signs(s), a, K, M, N)
+    assert np.max(np.abs(W.astype(np.float64) - Wk - RK.astype(np.float64))) <= 4 * 2.0 ** -24 * 0.2
+
+
+def test_residual_scale_rounds_once_from_fp64():
+    # Reading: the group mean is rounded once, fp64 -> fp16 nearest-even.
+    # Group: 126 x 1.0, 1 + 2^-4, 1 + 2^-23  ->  mean = 1 + 2^-11 + 2^-30,
+    # just above the fp16 midpoint 1 + 2^-11, so it rounds up to 1 + 2^-10;
+    # rounding through fp32 first would land on the midpoint and give 1.0.
+    assert np.float16(1 + 2.0 ** -11 + 2.0 ** -40) == np.float16(1 + 2.0 ** -10)
+    W = np.ones((1, 128), dtype=np.float32)
+    W[0, 5] = 1 + 2.0 ** -4
+    W[0, 77] = 1 + 2.0 ** -23
+    s, a, R = O.residual_binarize(W, 1)
+    assert a[0, 0, 0] == np.float16(1 + 2.0 ** -10)
+    assert np.float16(np.float32(1 + 2.0 ** -11 + 2.0 ** -30)) == np.float16(1.0)
+
+
+def test_residual_zero_group_and_sign_of_zero():
+    # sign(0) = +1 (also for -0.0); an all-zero group gets alpha = 0 and keeps R.
+    W = np.zeros((2, 256), dtype=np.float32)
+    W[0, 128:] = -0.0
+    W[1, :128] = np.linspace(-1, 1, 128, dtype=np.float32)
+    s, a, R = O.residual_binarize(W, 2)
+    assert (s[:, 0, :] == 1).all()
+    assert a[0, 0, 0] == 0 and a[0, 1, 0] == 0
+    assert np.array_equal(R[0], W[0])
+
+
+# --------------------------------------------------------------------------
+# Tolerance (O8)
+# --------------------------------------------------------------------------
+
+def test_tolerance_sanity():
+    K, M, N = 2, 32, 256
+    s, a, x = _signs_alpha_x(K, M, N, 80)
+    y, E = O.linear(O.pack_signs(s), a, K, M, N, x, "f32")
+    bound = 1e-3 * E + 1e-6
+    assert O.within_tolerance(y + 0.5 * bound, y, E).all()
+    assert not O.within_tolerance(y + 2.0 * bound, y, E).any()
+    assert O.rel_l2(y, y) == 0.0
