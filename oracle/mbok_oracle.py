@@ -41,15 +41,14 @@ Readings where the pages are silent (each one is listed in the design notes):
   value, as one fp32 subtraction;
   N must be a multiple of 128 (no ragged group).
 
-Bit layout "V1" (the pages give none; this is the library's storage format):
-  rows are cut into tiles of 128 (the last tile is padded; pad rows are
-  ignored), columns into groups of 128, each group into four 32-column chunks.
-  The packed array is a flat uint32 array ordered
-      [row tile rt][group g][row in tile r_in][chunk c][kernel k]
-  and bit i (least significant = 0) of a word holds column 128 g + 32 c + i.
-  So one row's record for one group is 4*K consecutive words, and for one
-  32-column chunk the K kernels' words sit side by side.
-Scales alpha are fp16 stored [M][N/128][K] (kernel index fastest).
+Storage format, version 1 (the pages give none; this is the library's format):
+  rows are cut into octets of 8 (the last octet is padded; pad rows are
+  ignored).  The packed kernels are bytes ordered
+      [octet o][kernel k][unit q][row i in octet][2 bytes]
+  where unit q covers columns 16q..16q+15: the little-endian 16-bit halfword
+  for row 8o+i holds column 16q+b in bit b.  A set bit means +1.
+  Scales alpha are fp16; logically [M][N/128][K], stored blocked as
+      [octet o][group g][kernel k][row i in octet].
 
 Parity pins: see tests/test_oracle_pins.py (brute force in exact rational
 arithmetic, flip invariance, level count, least-squares closed form, residual
@@ -63,40 +62,44 @@ import math
 import numpy as np
 
 GROUP = 128        # columns per scale group
-TILE_ROWS = 128    # rows per layout tile
-CHUNKS = GROUP // 32
+OCTET = 8          # rows per storage block
+UNIT = 16          # columns per 16-bit unit
 
 
 # --------------------------------------------------------------------------
-# Layout sizes and addressing (restated from the V1 definition above)
+# Layout sizes and addressing (restated from the format definition above)
 # --------------------------------------------------------------------------
 
 def n_groups(N: int) -> int:
-    if N % GROUP:
-        raise ValueError("N must be a multiple of 128")
+    if N % GROUP or N <= 0:
+        raise ValueError("N must be a positive multiple of 128")
     return N // GROUP
 
 
-def n_row_tiles(M: int) -> int:
-    return (M + TILE_ROWS - 1) // TILE_ROWS
+def n_octets(M: int) -> int:
+    return (M + OCTET - 1) // OCTET
 
 
-def packed_words(K: int, M: int, N: int) -> int:
-    return n_row_tiles(M) * n_groups(N) * TILE_ROWS * CHUNKS * K
+def packed_bytes(K: int, M: int, N: int) -> int:
+    n_groups(N)
+    return n_octets(M) * K * N
 
 
 def alpha_elems(K: int, M: int, N: int) -> int:
-    return M * n_groups(N) * K
+    return n_octets(M) * OCTET * n_groups(N) * K
 
 
-def word_and_bit(K: int, M: int, N: int, k: int, r: int, j: int) -> tuple[int, int]:
-    """Word index and bit position that hold kernel k, row r, column j."""
-    G = n_groups(N)
-    rt, r_in = divmod(r, TILE_ROWS)
-    g, jj = divmod(j, GROUP)
-    c, bit = divmod(jj, 32)
-    word = ((rt * G + g) * TILE_ROWS + r_in) * (CHUNKS * K) + c * K + k
-    return word, bit
+def byte_and_bit(K: int, M: int, N: int, k: int, r: int, j: int) -> tuple[int, int]:
+    """Byte offset and bit position that hold kernel k, row r, column j."""
+    o, i = divmod(r, OCTET)
+    q, b = divmod(j, UNIT)
+    byte = ((o * K + k) * (N // UNIT) + q) * UNIT + 2 * i + b // 8
+    return byte, b % 8
+
+
+def alpha_index(K: int, M: int, N: int, k: int, r: int, g: int) -> int:
+    o, i = divmod(r, OCTET)
+    return ((o * n_groups(N) + g) * K + k) * OCTET + i
 
 
 # --------------------------------------------------------------------------
@@ -104,33 +107,51 @@ def word_and_bit(K: int, M: int, N: int, k: int, r: int, j: int) -> tuple[int, i
 # --------------------------------------------------------------------------
 
 def pack_signs(signs: np.ndarray) -> np.ndarray:
-    """int8 signs [K][M][N] -> V1 words.  An entry >= 0 is stored as bit 1 (+1)."""
+    """int8 signs [K][M][N] -> packed bytes viewed as uint32 words.
+    An entry >= 0 is stored as a set bit (+1)."""
     K, M, N = signs.shape
-    G, RT = n_groups(N), n_row_tiles(M)
-    bits = np.zeros((K, RT * TILE_ROWS, N), dtype=np.uint64)
+    n_groups(N)
+    O = n_octets(M)
+    bits = np.zeros((K, O * OCTET, N), dtype=np.uint16)
     bits[:, :M, :] = signs >= 0
-    b = bits.reshape(K, RT, TILE_ROWS, G, CHUNKS, 32)
-    words = np.zeros((K, RT, TILE_ROWS, G, CHUNKS), dtype=np.uint64)
-    for i in range(32):
-        words |= b[..., i] << np.uint64(i)
-    # storage order [rt][g][r_in][c][k]
-    return np.ascontiguousarray(words.transpose(1, 3, 2, 4, 0)).astype(np.uint32).ravel()
+    b = bits.reshape(K, O, OCTET, N // UNIT, UNIT)
+    half = np.zeros((K, O, OCTET, N // UNIT), dtype=np.uint16)
+    for t in range(UNIT):
+        half |= b[..., t] << np.uint16(t)
+    # storage order [o][k][q][i], little-endian halfwords
+    h = np.ascontiguousarray(half.transpose(1, 0, 3, 2)).astype("<u2").ravel()
+    return h.view("<u4").astype(np.uint32)
 
 
 def unpack_rows(packed: np.ndarray, K: int, M: int, N: int, rows) -> np.ndarray:
-    """V1 words -> b in {-1,+1}, int8 [K][len(rows)][N], for the listed rows."""
-    G, RT = n_groups(N), n_row_tiles(M)
+    """Packed words -> b in {-1,+1}, int8 [K][len(rows)][N], for the listed rows."""
+    O = n_octets(M)
     rows = np.asarray(rows, dtype=np.int64)
-    w = np.asarray(packed, dtype=np.uint32).reshape(RT, G, TILE_ROWS, CHUNKS, K)
-    sel = w[rows // TILE_ROWS, :, rows % TILE_ROWS, :, :]          # [R][G][C][K]
-    shifts = np.arange(32, dtype=np.uint32)
-    bits = (sel[..., None] >> shifts) & np.uint32(1)                 # [R][G][C][K][32]
-    bits = bits.transpose(3, 0, 1, 2, 4).reshape(K, len(rows), N)   # [K][R][N]
+    h = np.ascontiguousarray(packed, dtype="<u4").view("<u2").reshape(O, K, N // UNIT, OCTET)
+    sel = h[rows // OCTET, :, :, rows % OCTET]                       # [R][K][N/16]
+    shifts = np.arange(UNIT, dtype=np.uint16)
+    bits = (sel[..., None] >> shifts) & np.uint16(1)                  # [R][K][N/16][16]
+    bits = bits.reshape(len(rows), K, N).transpose(1, 0, 2)           # [K][R][N]
     return np.where(bits == 1, 1, -1).astype(np.int8)
 
 
 def unpack_bits(packed: np.ndarray, K: int, M: int, N: int) -> np.ndarray:
     return unpack_rows(packed, K, M, N, np.arange(M))
+
+
+def block_alpha(alpha_mgk: np.ndarray, K: int, M: int, N: int) -> np.ndarray:
+    """fp16 [M][G][K] -> the stored order [o][g][k][i] (pad rows 0)."""
+    G, O = n_groups(N), n_octets(M)
+    a = np.zeros((O * OCTET, G, K), dtype=np.float16)
+    a[:M] = np.asarray(alpha_mgk, dtype=np.float16).reshape(M, G, K)
+    return np.ascontiguousarray(a.reshape(O, OCTET, G, K).transpose(0, 2, 3, 1)).ravel()
+
+
+def unblock_alpha(alpha_blk: np.ndarray, K: int, M: int, N: int) -> np.ndarray:
+    """The stored order -> fp16 [M][G][K]."""
+    G, O = n_groups(N), n_octets(M)
+    a = np.asarray(alpha_blk, dtype=np.float16).reshape(O, G, K, OCTET).transpose(0, 3, 1, 2)
+    return np.ascontiguousarray(a.reshape(O * OCTET, G, K)[:M])
 
 
 # --------------------------------------------------------------------------

@@ -29,30 +29,43 @@ def _signs_alpha_x(K, M, N, seed, x_dtype="f32"):
 # --------------------------------------------------------------------------
 
 def test_layout_hand_worked_example():
-    # tests/golden/layout_k2_1x128.txt: words derived by hand from the layout rules.
-    with open(os.path.join(GOLDEN, "layout_k2_1x128.txt")) as f:
+    # tests/golden/layout_k2_2x128.txt: words derived by hand from the format rules.
+    with open(os.path.join(GOLDEN, "layout_k2_2x128.txt")) as f:
         lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
-    assert lines[0] == "K=2 M=1 N=128"
-    expect = [int(t, 16) for t in lines[1].split()]
+    assert lines[0] == "K=2 M=2 N=128"
+    expect = [int(t, 16) for t in lines[1].split(":")[1].split()]
     j = np.arange(128)
-    signs = np.stack([np.where(j % 3 == 0, 1, -1), np.where(j < 40, 1, -1)]).astype(np.int8)[:, None, :]
+    signs = np.stack([
+        np.stack([np.where(j % 3 == 0, 1, -1), np.where((j == 5) | (j == 100), 1, -1)]),
+        np.stack([np.where(j < 40, 1, -1), -np.ones(128, dtype=int)]),
+    ]).astype(np.int8)                                  # [K=2][M=2][N=128]
     packed = O.pack_signs(signs)
-    assert packed.shape == (O.packed_words(2, 1, 128),) == (1024,)
-    assert [int(v) for v in packed[:8]] == expect
-    assert not packed[8:].any()
+    assert packed.shape == (O.packed_bytes(2, 2, 128) // 4,) == (64,)
+    assert [int(v) for v in packed[0::4]] == expect
+    assert not np.delete(packed, np.arange(0, 64, 4)).any()
+    idx = dict(t.split("=") for t in lines[2].split(":")[1].split())
+    for k in range(2):
+        for r in range(2):
+            assert O.alpha_index(2, 2, 128, k, r, 0) == int(idx[f"k{k}r{r}"])
+    assert O.alpha_elems(2, 2, 128) == int(idx["total"])
+    a = np.arange(4, dtype=np.float16).reshape(2, 1, 2)            # [M][G][K]
+    blk = O.block_alpha(a, 2, 2, 128)
+    assert blk.shape == (16,)
+    assert [float(blk[i]) for i in (0, 1, 8, 9)] == [0.0, 2.0, 1.0, 3.0]
+    assert np.array_equal(O.unblock_alpha(blk, 2, 2, 128), a)
 
 
 def test_layout_scalar_addressing_ragged():
-    # Vectorised packer agrees bit by bit with the scalar address rule, with a
-    # ragged last row tile (M=130) and three groups.
-    K, M, N = 3, 130, 384
+    # The vectorised packer agrees bit by bit with the scalar address rule, for
+    # a ragged last octet (M=13) and three groups.
+    K, M, N = 3, 13, 384
     s = wl.random_signs(K, M, N, 11, p_zero=0.05)
-    packed = O.pack_signs(s)
+    by = O.pack_signs(s).view(np.uint8)
     r = np.random.default_rng(5)
     for _ in range(3000):
         k, row, col = int(r.integers(K)), int(r.integers(M)), int(r.integers(N))
-        w, b = O.word_and_bit(K, M, N, k, row, col)
-        assert (int(packed[w]) >> b) & 1 == int(s[k, row, col] >= 0)
+        byte, bit = O.byte_and_bit(K, M, N, k, row, col)
+        assert (int(by[byte]) >> bit) & 1 == int(s[k, row, col] >= 0)
 
 
 def test_layout_round_trip_and_zero_maps_to_plus_one():
@@ -60,6 +73,8 @@ def test_layout_round_trip_and_zero_maps_to_plus_one():
     s = wl.random_signs(K, M, N, 12, p_zero=0.1)
     b = O.unpack_bits(O.pack_signs(s), K, M, N)
     assert np.array_equal(b, np.where(s >= 0, 1, -1))
+    a = wl.alpha_decaying(K, M, N, 13)
+    assert np.array_equal(O.unblock_alpha(O.block_alpha(a, K, M, N), K, M, N), a)
 
 
 # --------------------------------------------------------------------------
