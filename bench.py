@@ -1,0 +1,482 @@
+#!/usr/bin/env python3
+"""Benchmark of the MBOK linear layer on B200.
+
+Headline: packed-weight HBM GB/s (and us/layer) of the K=3 Boolean decode
+GEMV on the LLaMA-7B q_proj shape (M = N = 4096, group 128, batch 1, bf16 x).
+One step is one decode pass over L distinct weight copies of that shape
+(L = 48 by default: 340 MB of packed weights, well above the 126 MB L2, so
+every launch reads its weights from HBM).  The step is captured once in a
+CUDA graph and replayed; time is taken with CUDA events on the launching
+stream, max over ranks when several GPUs run replicas.
+
+Also reported on the same JSON line: the roofline of the GEMV kernel, an
+end-to-end number through the C ABI with host buffers, the CPU oracle
+baseline, SM clocks sampled during the timed region, and secondary rows
+(prefill GEMM, small batch, the LLaMA-13B layer sweep, residual
+binarisation, packing).
+
+`--impl reference` times the CPU oracle (the correctness reference of this
+repository) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "packed-weight HBM GB/s (% of peak) and us/layer, K-kernel Boolean GEMV/GEMM"
+UNIT = "GB/s"
+
+
+def args_parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["mbok", "reference"], default="mbok")
+    p.add_argument("--layers", type=int, default=48, help="distinct weight copies per step")
+    p.add_argument("--no-extras", action="store_true", help="skip the secondary rows")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "boolean_weight_matmul_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_file: str, key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(key)
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_rate(seconds: float = 10.0):
+    """The oracle as it stands: packed-weight GB/s of oracle.linear on sampled
+    rows of one q_proj layer, repeated for about `seconds`."""
+    from oracle import mbok_oracle as O
+    from boolean_weight_matmul_b200 import workloads as wl
+    K, M, N = 3, 4096, 4096
+    words = wl.random_words(O.packed_bytes(K, M, N) // 4, wl.seed_of(2, 0, 0))
+    a = wl.alpha_decaying(K, M, N, wl.seed_of(2, 0, 1))
+    x = wl.x_normal(1, N, wl.seed_of(2, 0, 2))
+    rows_per_call = 256
+    bytes_per_row = K * N / 8 + 2 * K * N / 128
+    t0 = time.perf_counter()
+    n_rows = 0
+    calls = 0
+    rng = np.random.default_rng(0)
+    while time.perf_counter() - t0 < seconds:
+        rows = np.sort(rng.choice(M, rows_per_call, replace=False))
+        O.linear(words, a, K, M, N, x, "bf16", rows=rows)
+        n_rows += rows_per_call
+        calls += 1
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return {"value": n_rows * bytes_per_row / dt / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{calls} calls of oracle.linear on {rows_per_call} random rows of one K=3 "
+                      f"4096x4096 layer ({n_rows} rows, {dt:.1f} s); numpy fp64"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(max(0, a.warmup)):
+        cpu_oracle_rate(0.5)
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(a.steps):
+        last = cpu_oracle_rate(1.0)
+        vals.append(last["value"])
+    dt = time.perf_counter() - t0
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * dt / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "llama7b_q_proj_k3_4096x4096_gemv_b1", "K": 3, "M": 4096,
+                       "N": 4096, "group": 128, "batch": 1,
+                       "sample": "each step: 1 s of oracle.linear on 256 random rows"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def build_layers(torch, mb, wl, K, M, N, L, dev, seed0):
+    """L distinct packed weights (random words = Bernoulli(0.5) bits) with
+    decaying scales, plus L activation vectors."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed0)
+    nb = mb.packed_bytes(K, M, N)
+    packed = [torch.randint(-2 ** 31, 2 ** 31 - 1, (nb // 4,), dtype=torch.int32, device=dev, generator=g)
+              for _ in range(L)]
+    alphas = []
+    for l in range(L):
+        a = wl.alpha_decaying(K, M, N, seed0 + 10 * l + 1)
+        ad = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.float16)
+        out = mb.empty_alpha(K, M, N, dev)
+        mb.pack_alpha(ad, K, M, N, out)
+        alphas.append(out)
+    xs = [torch.from_numpy(wl.x_normal(1, N, seed0 + 10 * l + 2).view(np.int16)).to(dev).view(torch.bfloat16)
+          for l in range(L)]
+    return packed, alphas, xs
+
+
+def time_graph(torch, fn, steps, warmup, stream):
+    """Capture fn() once, replay warmup + steps times; returns ms per replay."""
+    with torch.cuda.stream(stream):
+        fn()   # eager warm-up (sets kernel attributes outside capture)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        fn()
+    # replay() launches on the current stream: make it the captured stream so
+    # the events bracket the replays.
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps, graph
+
+
+def run_gpu(a):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    from boolean_weight_matmul_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        mbuild.build()
+    if world > 1:
+        dist.barrier()
+    peaks, peak_src = measured_peaks()
+
+    # CPU baseline first (rank 0, N=1 only), before any GPU work is timed.
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_oracle_rate(10.0)
+
+    K, M, N, L = 3, 4096, 4096, a.layers
+    bytes_per_layer = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
+    packed, alphas, xs = build_layers(torch, mb, wl, K, M, N, L, dev, 1000 * 2 + 7919 * rank)
+    ws = mb.zeros_workspace(K, M, N, 1, dev)
+    ys = [torch.empty(1, M, dtype=torch.float32, device=dev) for _ in range(L)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        for l in range(L):
+            mb.gemv(packed[l], alphas[l], K, M, N, 128, xs[l], mb.BF16, 1, ys[l], ws, stream=stream)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        ms, graph = time_graph(torch, step, a.steps, a.warmup, stream)
+    clocks = clk.summary()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    value = world * L * bytes_per_layer / (ms * 1e-3) / 1e9
+    us_per_layer = 1e3 * ms / L
+    achieved = bytes_per_layer / (us_per_layer * 1e-6) / 1e9
+    traffic = ncu_traffic("gemv_lut.cu", "gemv_lut8_q_proj_k3_4096x4096")
+
+    # End to end through the C ABI with host buffers: per step, copy the L
+    # activation vectors host->device, run the L GEMVs, copy the L outputs back.
+    x_host = torch.stack([x.view(torch.int16).cpu() for x in xs]).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    y_host = torch.empty(L, M, dtype=torch.float32).pin_memory()
+    y_dev = torch.empty(L, M, dtype=torch.float32, device=dev)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        for l in range(L):
+            mb.gemv(packed[l], alphas[l], K, M, N, 128, x_dev[l].view(torch.bfloat16), mb.BF16, 1,
+                    y_dev[l], ws, stream=stream)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / a.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * L * bytes_per_layer / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+           "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
+           "ms_per_step": e2e_ms, "path": "mbok_gemv via the C ABI, pinned host x/y, copies in the timed region"}
+
+    del graph
+    extras = None
+    if not a.no_extras:
+        del packed, alphas, xs, ys
+        torch.cuda.empty_cache()
+        extras = run_extras(torch, mb, wl, dev, peaks, a)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x, 1-bit kernels, fp16 scales, fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": "llama7b_q_proj_k3_4096x4096_gemv_b1", "K": K, "M": M, "N": N,
+                   "group": 128, "batch": 1, "layers_per_step": L,
+                   "bytes_per_layer": bytes_per_layer, "us_per_layer": us_per_layer,
+                   "l2": f"inputs larger than L2: {L} distinct weight copies, "
+                         f"{L * bytes_per_layer / 1e6:.0f} MB per step vs 126 MB L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "gemv_lut8_kernel<3,false>",
+                     "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
+                     else "fallback 6.65 TB/s"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": a.steps * L,
+        "rows": extras,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_extras(torch, mb, wl, dev, peaks, a):
+    """Secondary rows, each timed with CUDA events (graph replays)."""
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(12345)
+
+    # Prefill GEMM, K=3, 4096 x 4096, 2048 tokens.
+    K, M, N, T = 3, 4096, 4096, 2048
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                           device=dev, generator=g)
+    alpha = mb.empty_alpha(K, M, N, dev)
+    mb.pack_alpha(torch.from_numpy(wl.alpha_decaying(K, M, N, 4001).view(np.int16)).to(dev).view(torch.float16),
+                  K, M, N, alpha)
+    X = torch.randn(T, N, device=dev, generator=g).to(torch.bfloat16)
+    Y = torch.empty(T, M, dtype=torch.bfloat16, device=dev)
+    ms, gr = time_graph(torch, lambda: mb.gemm(packed, alpha, K, M, N, 128, X, T, Y, stream=stream),
+                        10, 3, stream)
+    tflops = 2.0 * M * N * T / (ms * 1e-3) / 1e12
+    out["prefill_gemm_llama7b_q_proj_k3_t2048"] = {
+        "us": 1e3 * ms, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+        "peak_tflops": peaks["bf16_tflops"], "kernel": "gemm_mma_kernel"}
+    del gr, packed, X, Y
+    torch.cuda.empty_cache()
+
+    # Small batch, LLaMA-7B gate 11008 x 4096, K=3 (and down 4096 x 11008, K=2).
+    for (name, K, M, N) in (("gate", 3, 11008, 4096), ("down", 2, 4096, 11008)):
+        L = 8
+        packed = [torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                                device=dev, generator=g) for _ in range(L)]
+        al = []
+        for l in range(L):
+            t = mb.empty_alpha(K, M, N, dev)
+            mb.pack_alpha(torch.from_numpy(wl.alpha_decaying(K, M, N, 5000 + l).view(np.int16)).to(dev)
+                          .view(torch.float16), K, M, N, t)
+            al.append(t)
+        ws = mb.zeros_workspace(K, M, N, 16, dev)
+        bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
+        for batch in (1, 4, 16):
+            x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
+            y = torch.empty(batch, M, dtype=torch.float32, device=dev)
+
+            def fn():
+                for l in range(L):
+                    mb.gemv(packed[l], al[l], K, M, N, 128, x, mb.BF16, batch, y, ws, stream=stream)
+            ms, gr = time_graph(torch, fn, 10, 3, stream)
+            gbs = L * bpl / (ms * 1e-3) / 1e9
+            out[f"gemv_llama7b_{name}_k{K}_{M}x{N}_b{batch}"] = {
+                "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+            del gr
+        del packed, al
+        torch.cuda.empty_cache()
+
+    # LLaMA-13B linear sweep, K=4, 40 layers x 7 matrices, batch 1.
+    K = 4
+    layers = wl.LLAMA13B_LAYERS
+    mats = []
+    total_bytes = 0
+    for _ in range(layers):
+        for (name, M, N) in wl.LLAMA13B_LAYER:
+            p = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                              device=dev, generator=g)
+            al = torch.empty(mb.alpha_elems(K, M, N), dtype=torch.float16, device=dev)
+            al.copy_((torch.rand(al.shape, device=dev, generator=g) + 0.5) * 0.01)
+            mats.append((p, al, M, N))
+            total_bytes += mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
+    ws = mb.zeros_workspace(K, 13824, 13824, 1, dev)
+    xin = {N: torch.randn(1, N, device=dev, generator=g).to(torch.bfloat16) for N in (5120, 13824)}
+    yout = {M: torch.empty(1, M, dtype=torch.float32, device=dev) for M in (5120, 13824)}
+
+    def sweep():
+        for (p, al, M, N) in mats:
+            mb.gemv(p, al, K, M, N, 128, xin[N], mb.BF16, 1, yout[M], ws, stream=stream)
+    ms, gr = time_graph(torch, sweep, 5, 2, stream)
+    gbs = total_bytes / (ms * 1e-3) / 1e9
+    out["sweep_llama13b_k4_40x7_b1"] = {"ms_per_token": ms, "tokens_per_s": 1e3 / ms,
+                                       "bytes_per_token": total_bytes, "gbs": gbs,
+                                       "frac_of_hbm": gbs / peaks["hbm_gbs"], "launches": len(mats)}
+    del gr, mats
+    torch.cuda.empty_cache()
+
+    # Residual binarisation, LLaMA-7B gate 11008 x 4096, K=3.
+    K, M, N = 3, 11008, 4096
+    W = torch.randn(M, N, device=dev, generator=g) * 0.02
+    packed = mb.empty_packed(K, M, N, dev)
+    alpha = mb.empty_alpha(K, M, N, dev)
+    R = torch.empty_like(W)
+    ms, gr = time_graph(torch, lambda: mb.residual_binarize(W, M, N, K, 128, packed, alpha, R, stream=stream),
+                        5, 2, stream)
+    out["residual_binarize_llama7b_gate_k3"] = {"ms": ms, "gbs_of_w": 2 * W.numel() * 4 / (ms * 1e-3) / 1e9}
+    del gr
+    # Packing of int8 signs, same shape.
+    S = torch.randint(-1, 1, (K, M, N), dtype=torch.int8, device=dev, generator=g)
+    ms, gr = time_graph(torch, lambda: mb.pack_bits(S, K, M, N, packed, stream=stream), 5, 2, stream)
+    out["pack_bits_llama7b_gate_k3"] = {"ms": ms, "gbs_in": S.numel() / (ms * 1e-3) / 1e9}
+    del gr
+    return out
+
+
+def main():
+    a = args_parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_gpu(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+"""Python binding of libmbok, the B200 library for the multi-Boolean-kernel
+(MBOK) linear layer y = W x with W = sum_k alpha_k * B_k.
+
+This module only marshals arguments: every call below forwards device
+pointers, sizes and the current CUDA stream to the C ABI declared in
+include/mbok.h, where all work runs in the library's kernels.  There is no
+CPU fallback: a missing library or a CPU tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmbok.so")
+
+OK = 0
+F32 = 0
+BF16 = 1
+GROUP = 128
+MAX_K = 4
+MAX_BATCH = 16
+
+_lib = None
+
+
+class MbokError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmbok.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m boolean_weight_matmul_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        sigs = {
+            "mbok_status_string": ([i], ctypes.c_char_p),
+            "mbok_layout_version": ([], i),
+            "mbok_packed_bytes": ([i, i, i], sz),
+            "mbok_alpha_elems": ([i, i, i], sz),
+            "mbok_gemv_workspace_bytes": ([i, i, i, i], sz),
+            "mbok_pack_bits": ([vp, i, i, i, vp, vp], i),
+            "mbok_pack_alpha": ([vp, i, i, i, vp, vp], i),
+            "mbok_residual_binarize": ([vp, i, i, i, i, vp, vp, vp, vp], i),
+            "mbok_gemv": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp], i),
+            "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
+        }
+        for name, (args, res) in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mbok_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise MbokError(what, status)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("MBOK operates on CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("MBOK needs contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# ---- sizes ---------------------------------------------------------------
+
+def layout_version() -> int:
+    return lib().mbok_layout_version()
+
+
+def packed_bytes(K: int, M: int, N: int) -> int:
+    return lib().mbok_packed_bytes(K, M, N)
+
+
+def alpha_elems(K: int, M: int, N: int) -> int:
+    return lib().mbok_alpha_elems(K, M, N)
+
+
+def gemv_workspace_bytes(K: int, M: int, N: int, batch: int = 1) -> int:
+    return lib().mbok_gemv_workspace_bytes(K, M, N, batch)
+
+
+# ---- allocation helpers (torch owns the memory) --------------------------
+
+def empty_packed(K: int, M: int, N: int, device="cuda") -> torch.Tensor:
+    n = packed_bytes(K, M, N)
+    if n == 0:
+        raise MbokError("packed_bytes", 2)
+    return torch.empty(n // 4, dtype=torch.int32, device=device)
+
+
+def empty_alpha(K: int, M: int, N: int, device="cuda") -> torch.Tensor:
+    n = alpha_elems(K, M, N)
+    if n == 0:
+        raise MbokError("alpha_elems", 2)
+    return torch.empty(n, dtype=torch.float16, device=device)
+
+
+def zeros_workspace(K: int, M: int, N: int, batch: int = 1, device="cuda") -> torch.Tensor:
+    n = max(gemv_workspace_bytes(K, M, N, batch), 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+# ---- the calls ------------------------------------------------------------
+
+def pack_bits(signs, K, M, N, packed, stream=None) -> None:
+    _check(lib().mbok_pack_bits(_ptr(signs), K, M, N, _ptr(packed), _stream(stream)), "mbok_pack_bits")
+
+
+def pack_alpha(alpha_mgk, K, M, N, alpha_out, stream=None) -> None:
+    _check(lib().mbok_pack_alpha(_ptr(alpha_mgk), K, M, N, _ptr(alpha_out), _stream(stream)),
+           "mbok_pack_alpha")
+
+
+def residual_binarize(W, M, N, K, group, packed, alpha, residual=None, stream=None) -> None:
+    _check(lib().mbok_residual_binarize(_ptr(W), M, N, K, group, _ptr(packed), _ptr(alpha),
+                                        _ptr(residual), _stream(stream)), "mbok_residual_binarize")
+
+
+def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=None) -> None:
+    ws_bytes = 0 if workspace is None else (workspace.numel() * workspace.element_size()
+                                            if isinstance(workspace, torch.Tensor) else 0)
+    _check(lib().mbok_gemv(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype, batch,
+                           _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv")
+
+
+def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:
+    _check(lib().mbok_gemm(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(X), T, _ptr(Y),
+                           _stream(stream)), "mbok_gemm")
+
+
+def dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.float32:
+        return F32
+    if x.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported activation dtype {x.dtype}")

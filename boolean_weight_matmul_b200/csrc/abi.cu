@@ -1,0 +1,148 @@
+// C ABI of the MBOK library: argument checks on the host, then launches on
+// the caller's stream.  Nothing here allocates, synchronises or keeps state
+// beyond cached kernel attributes.
+#include "mbok_common.cuh"
+
+namespace mbok {
+cudaError_t launch_pack_bits(const int8_t*, const Shape&, uint8_t*, cudaStream_t);
+cudaError_t launch_pack_alpha(const uint16_t*, const Shape&, uint16_t*, cudaStream_t);
+cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __half*, float*,
+                                     cudaStream_t);
+cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
+                            float*, void*, cudaStream_t);
+size_t gemv_lut_workspace_bytes(const Shape&);
+cudaError_t launch_gemm_mma(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
+                            uint16_t*, float*, cudaStream_t);
+}  // namespace mbok
+
+using namespace mbok;
+
+namespace {
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Common shape checks; returns MBOK_OK or the first failing status.
+int check_shape(int K, int M, int N) {
+  if (K < 1 || K > MBOK_MAX_K) return MBOK_ERR_INVALID_ARG;
+  if (M < 1 || N < MBOK_GROUP || N % MBOK_GROUP != 0) return MBOK_ERR_SHAPE;
+  // keep every grid dimension and 32-bit unit index in range
+  if (M > (1 << 22) || N > (1 << 20)) return MBOK_ERR_SHAPE;
+  return MBOK_OK;
+}
+
+inline int from_cuda(cudaError_t e) { return e == cudaSuccess ? MBOK_OK : MBOK_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mbok_status_string(int status) {
+  switch (status) {
+    case MBOK_OK: return "ok";
+    case MBOK_ERR_INVALID_ARG: return "invalid argument";
+    case MBOK_ERR_SHAPE: return "unsupported shape";
+    case MBOK_ERR_ALIGN: return "misaligned pointer";
+    case MBOK_ERR_UNSUPPORTED: return "unsupported option";
+    case MBOK_ERR_CUDA: return "CUDA launch error";
+    case MBOK_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int mbok_layout_version(void) { return MBOK_LAYOUT_VERSION; }
+
+size_t mbok_packed_bytes(int K, int M, int N) {
+  if (check_shape(K, M, N) != MBOK_OK) return 0;
+  const Shape s = make_shape(K, M, N);
+  return size_t(s.O) * K * N;
+}
+
+size_t mbok_alpha_elems(int K, int M, int N) {
+  if (check_shape(K, M, N) != MBOK_OK) return 0;
+  const Shape s = make_shape(K, M, N);
+  return size_t(s.O) * kOctet * s.G * K;
+}
+
+size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch) {
+  if (check_shape(K, M, N) != MBOK_OK || batch < 1 || batch > MBOK_MAX_BATCH) return 0;
+  return gemv_lut_workspace_bytes(make_shape(K, M, N));
+}
+
+int mbok_pack_bits(const int8_t* signs, int K, int M, int N, uint32_t* packed, void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (signs == nullptr || packed == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(signs, 16) || !aligned(packed, 16)) return MBOK_ERR_ALIGN;
+  return from_cuda(launch_pack_bits(signs, make_shape(K, M, N), reinterpret_cast<uint8_t*>(packed),
+                                    as_stream(stream)));
+}
+
+int mbok_pack_alpha(const uint16_t* alpha_mgk, int K, int M, int N, uint16_t* alpha_out,
+                    void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (alpha_mgk == nullptr || alpha_out == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(alpha_mgk, 16) || !aligned(alpha_out, 16)) return MBOK_ERR_ALIGN;
+  return from_cuda(launch_pack_alpha(alpha_mgk, make_shape(K, M, N), alpha_out, as_stream(stream)));
+}
+
+int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint32_t* packed,
+                           uint16_t* alpha, float* residual, void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (W == nullptr || packed == nullptr || alpha == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(alpha, 16) ||
+      (residual != nullptr && !aligned(residual, 16)))
+    return MBOK_ERR_ALIGN;
+  const Shape s = make_shape(K, M, N);
+  if (s.O > 65535) return MBOK_ERR_SHAPE;
+  return from_cuda(launch_residual_binarize(W, s, reinterpret_cast<uint8_t*>(packed),
+                                            reinterpret_cast<__half*>(alpha), residual,
+                                            as_stream(stream)));
+}
+
+int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const void* x, int x_dtype, int batch, float* y, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (packed == nullptr || alpha == nullptr || x == nullptr || y == nullptr)
+    return MBOK_ERR_INVALID_ARG;
+  if (x_dtype != MBOK_F32 && x_dtype != MBOK_BF16) return MBOK_ERR_INVALID_ARG;
+  if (batch < 1 || batch > MBOK_MAX_BATCH) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(x, 16) || !aligned(y, 4))
+    return MBOK_ERR_ALIGN;
+  const Shape s = make_shape(K, M, N);
+  const size_t need = gemv_lut_workspace_bytes(s);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
+    return MBOK_ERR_WORKSPACE;
+  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
+    const cudaError_t e = launch_gemv_lut(reinterpret_cast<const uint8_t*>(packed), alpha, s, xb,
+                                          x_dtype == MBOK_F32, y + size_t(b) * M, workspace,
+                                          as_stream(stream));
+    if (e != cudaSuccess) return MBOK_ERR_CUDA;
+  }
+  return MBOK_OK;
+}
+
+int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const uint16_t* X, int T, uint16_t* Y, void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (T < 1 || T > (1 << 24)) return MBOK_ERR_SHAPE;
+  if (packed == nullptr || alpha == nullptr || X == nullptr || Y == nullptr)
+    return MBOK_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(X, 16) || !aligned(Y, 16))
+    return MBOK_ERR_ALIGN;
+  return from_cuda(launch_gemm_mma(reinterpret_cast<const uint8_t*>(packed), alpha,
+                                   make_shape(K, M, N), X, T, Y, nullptr, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+/*
+ * mbok.h - C ABI of the multi-Boolean-kernel (MBOK) linear layer on B200.
+ *
+ * The method ("Highly Efficient and Effective LLMs with Multi-Boolean
+ * Architectures", ICLR 2026) stores a weight matrix as K Boolean kernels with
+ * group-wise scales,
+ *
+ *     W[r][j] = sum_{k<K} alpha[k][r][g(j)] * B_k[r][j],   B_k in {-1,+1},
+ *     g(j) = j / 128,
+ *
+ * (Paper-Notes page, section 方法详解 / 关键设计: multi-kernel Boolean
+ * parameters, group-wise scaling with groups of 128) and evaluates y = W x as
+ * K Boolean matrix-vector products (same section).
+ *
+ * Conventions for every call
+ *  - All data pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates nothing, keeps no state between calls and never synchronises.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued on it; results are ready when the stream reaches them.
+ *  - Return value: an mbok_status.  Argument errors are detected on the host
+ *    and returned before anything is launched; a launch error returns
+ *    MBOK_ERR_CUDA.  No call aborts, traps or throws.
+ *  - Group size: `group` arguments must equal MBOK_GROUP (128); N must be a
+ *    positive multiple of 128.  1 <= K <= MBOK_MAX_K.  M >= 1.
+ *
+ * Storage format MBOK_LAYOUT_VERSION 1 (the pages define none):
+ *  - Rows are cut into octets of 8 (O = ceil(M/8); rows of the last octet at
+ *    or beyond M are padding and are ignored by every reader).
+ *  - packed: O*K*N bits as bytes ordered [octet o][kernel k][unit q][row i][2],
+ *    where unit q holds columns 16q..16q+15 of rows 8o..8o+7 in 16 bytes:
+ *    the 16-bit little-endian halfword i of the unit is row 8o+i, and its bit b
+ *    is column 16q+b.  A set bit means +1, a clear bit means -1.
+ *  - alpha: fp16 (IEEE binary16 bit patterns) ordered [octet o][group g]
+ *    [kernel k][row i], i.e. element ((o*G + g)*K + k)*8 + i is the scale of
+ *    kernel k, row 8o+i, group g (G = N/128).  Pad rows are ignored.
+ *  - packed must be 16-byte aligned, alpha 16-byte aligned.
+ */
+#ifndef MBOK_H
+#define MBOK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MBOK_OK = 0,
+  MBOK_ERR_INVALID_ARG = 1,   /* NULL pointer, K / batch / dtype out of range */
+  MBOK_ERR_SHAPE = 2,         /* M < 1, N not a positive multiple of 128, T < 1 */
+  MBOK_ERR_ALIGN = 3,         /* a pointer lacks its required alignment */
+  MBOK_ERR_UNSUPPORTED = 4,   /* group != 128 */
+  MBOK_ERR_CUDA = 5,          /* a kernel launch failed */
+  MBOK_ERR_WORKSPACE = 6      /* workspace NULL or smaller than required */
+} mbok_status;
+
+typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
+
+#define MBOK_GROUP 128
+#define MBOK_LAYOUT_VERSION 1
+#define MBOK_MAX_K 4
+#define MBOK_MAX_BATCH 16
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mbok_status_string(int status);
+
+/* The storage-format version this library reads and writes (1). */
+int mbok_layout_version(void);
+
+/* Bytes of the packed kernels for (K, M, N): ceil(M/8)*K*N.  0 on bad shape. */
+size_t mbok_packed_bytes(int K, int M, int N);
+
+/* fp16 elements of the blocked scales: ceil(M/8)*8*(N/128)*K.  0 on bad shape. */
+size_t mbok_alpha_elems(int K, int M, int N);
+
+/* Bytes of device workspace mbok_gemv needs for (K, M, N, batch).  The caller
+ * allocates it (256-byte aligned), zero-fills it ONCE before its first use,
+ * and may reuse it for any later call with the same or smaller requirement
+ * on the same stream; calls leave it zero-filled where that matters.  Calls
+ * that share one workspace must not run concurrently. */
+size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch);
+
+/* Pack K sign matrices into layout 1.
+ *   signs  : int8 [K][M][N], row-major; an entry >= 0 means +1 (so 0 -> +1),
+ *            an entry < 0 means -1.  (B_k in {-1,+1}: Paper-Notes 关键设计.)
+ *   packed : mbok_packed_bytes(K,M,N) bytes, 16-byte aligned; every byte is
+ *            written (pad rows as 0 bits). */
+int mbok_pack_bits(const int8_t* signs, int K, int M, int N, uint32_t* packed, void* stream);
+
+/* Reorder scales from the logical fp16 [M][N/128][K] (kernel fastest) into
+ * the blocked order of layout 1.  alpha_out holds mbok_alpha_elems(K,M,N)
+ * elements; pad rows are written as 0.  Both pointers 16-byte aligned. */
+int mbok_pack_alpha(const uint16_t* alpha_mgk, int K, int M, int N, uint16_t* alpha_out,
+                    void* stream);
+
+/* Greedy residual binarisation, producing K kernels from a dense weight.
+ * Each later kernel fits the residual the earlier ones leave (Dutch and
+ * Spanish technical summaries, "Successive SVID" / "Extracción Sucesiva");
+ * for a fixed sign matrix the least-squares group scale is mean|R|
+ * (Paper-Notes 关键设计, closed-form scale).  Per row r and group g,
+ * for k = 0..K-1:
+ *     b      = sign(R) with sign(0) = +1 (also for -0.0),
+ *     alpha  = fp16( (sum over the group's 128 columns of |R|, accumulated in
+ *              fp64 in column order) / 128 ), rounded once, nearest-even,
+ *     R      = R - alpha*b   (fp32, with the fp16 alpha, one rounding),
+ * starting from R = W.  Results are bit-exact and deterministic.
+ *   W        : fp32 [M][N] row-major (16-byte aligned).
+ *   packed   : layout 1, mbok_packed_bytes(K,M,N) bytes.
+ *   alpha    : layout 1, mbok_alpha_elems(K,M,N) fp16 elements.
+ *   residual : fp32 [M][N] receiving R after the K-th kernel, or NULL.
+ * NaN in W yields unspecified bits and NaN scales for its group. */
+int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint32_t* packed,
+                           uint16_t* alpha, float* residual, void* stream);
+
+/* y[b][r] = sum_j W[r][j] * x[b][j] for b < batch (decode / small batch).
+ * Evaluated as sum over groups and kernels of alpha[k][r][g] times the
+ * +-1 dot product of B_k's group slice with x (Paper-Notes 关键设计: Wx as
+ * K Boolean matrix-vector products), accumulated in fp32.
+ *   packed, alpha : layout 1.
+ *   x       : [batch][N], fp32 (x_dtype MBOK_F32) or bf16 bit patterns
+ *             (MBOK_BF16); 16-byte aligned.
+ *   batch   : 1..MBOK_MAX_BATCH.
+ *   y       : fp32 [batch][M] (4-byte aligned), fully overwritten.
+ *   workspace, workspace_bytes : see mbok_gemv_workspace_bytes.
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_j |W[r][j] x[b][j]| + 1e-6 per
+ * element and relative L2 error <= 1e-5 (fp32 accumulation).  For a given
+ * (shape, batch) the result is deterministic run to run. */
+int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const void* x, int x_dtype, int batch, float* y, void* workspace,
+              size_t workspace_bytes, void* stream);
+
+/* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill), where Wt is W
+ * rounded to bf16 element-wise, multiplied on the tensor cores with fp32
+ * accumulation, and Y is rounded to bf16.  X: bf16 [T][N]; Y: bf16 [T][M];
+ * both 16-byte aligned.  Accuracy: |Y - Y_exact| <= 1e-3 * sum_j |W x| + 1e-6
+ * per element (bf16 weight and output rounding). */
+int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const uint16_t* X, int T, uint16_t* Y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MBOK_H */

@@ -1,0 +1,83 @@
+"""Shared helpers for the MBOK tests (device buffers, oracle comparisons)."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import mbok_oracle as O
+
+GEMV_REL = 1e-3
+GEMV_ABS = 1e-6
+GEMV_REL_L2 = 1e-5
+
+
+def ensure_built():
+    from boolean_weight_matmul_b200 import build
+    return build.build()
+
+
+def to_dev(a: np.ndarray):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.cuda()
+
+
+def packed_from_signs_gpu(signs: np.ndarray):
+    """GPU packing (the product) of int8 signs [K][M][N]."""
+    import boolean_weight_matmul_b200 as mb
+    K, M, N = signs.shape
+    packed = mb.empty_packed(K, M, N)
+    mb.pack_bits(to_dev(signs), K, M, N, packed)
+    return packed
+
+
+def alpha_blocked_gpu(alpha_mgk: np.ndarray, K: int, M: int, N: int):
+    """GPU blocking (the product) of logical fp16 scales [M][G][K]."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    a = to_dev(np.ascontiguousarray(alpha_mgk, dtype=np.float16).view(np.int16)).view(torch.float16)
+    out = mb.empty_alpha(K, M, N)
+    mb.pack_alpha(a, K, M, N, out)
+    return out
+
+
+def x_dev(x: np.ndarray, dtype: str):
+    import torch
+    if dtype == "f32":
+        return to_dev(x.astype(np.float32))
+    return to_dev(x.view(np.int16)).view(torch.bfloat16)
+
+
+def gemv_gpu(packed, alpha_blk, K, M, N, x_np, x_dtype):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    batch = x_np.shape[0]
+    x = x_dev(x_np, x_dtype)
+    y = torch.empty(batch, M, dtype=torch.float32, device="cuda")
+    ws = mb.zeros_workspace(K, M, N, batch)
+    mb.gemv(packed, alpha_blk, K, M, N, 128, x, mb.F32 if x_dtype == "f32" else mb.BF16, batch, y, ws)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def gemm_gpu(packed, alpha_blk, K, M, N, X_bits: np.ndarray):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    T = X_bits.shape[0]
+    X = x_dev(X_bits, "bf16")
+    Y = torch.empty(T, M, dtype=torch.bfloat16, device="cuda")
+    mb.gemm(packed, alpha_blk, K, M, N, 128, X, T, Y)
+    torch.cuda.synchronize()
+    return Y.float().cpu().numpy()
+
+
+def assert_close(y, y_ref, E, rel_l2=None, what=""):
+    """Per-element |y - y_ref| <= 1e-3 E + 1e-6, and optionally rel-L2."""
+    ok = O.within_tolerance(y, y_ref, E, GEMV_REL, GEMV_ABS)
+    if not ok.all():
+        bad = np.argwhere(~ok)[:5]
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements out of tolerance, e.g. "
+                             + ", ".join(f"{tuple(b)} got {float(y[tuple(b)])} want {float(y_ref[tuple(b)])} "
+                                         f"bound {GEMV_REL * float(E[tuple(b)]) + GEMV_ABS}" for b in bad))
+    if rel_l2 is not None:
+        e = O.rel_l2(y, y_ref)
+        assert e <= rel_l2, f"{what}: relative L2 error {e} > {rel_l2}"

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU work): the library loads, exports
+every function include/mbok.h declares, sizes are right, and argument errors
+are reported before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from helpers import ensure_built
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mbok.h")
+
+FAKE = 1 << 20          # a 16-byte aligned non-null address; never dereferenced
+FAKE_ODD = FAKE + 1     # misaligned
+
+
+@pytest.fixture(scope="module")
+def L():
+    ensure_built()
+    import boolean_weight_matmul_b200 as mb
+    return mb.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^\s*(?:const\s+char\s*\*|int|size_t)\s+(mbok_\w+)\s*\(", text, re.M)
+
+
+def test_header_declares_the_calls():
+    names = set(header_functions())
+    for n in ("mbok_pack_bits", "mbok_residual_binarize", "mbok_gemv", "mbok_gemm",
+              "mbok_pack_alpha", "mbok_packed_bytes", "mbok_alpha_elems",
+              "mbok_gemv_workspace_bytes", "mbok_status_string", "mbok_layout_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function(L):
+    names = header_functions()
+    assert names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/mbok.h but not exported"
+
+
+def test_sizes(L):
+    assert L.mbok_layout_version() == 1
+    assert L.mbok_packed_bytes(3, 4096, 4096) == 512 * 3 * 4096
+    assert L.mbok_packed_bytes(1, 13, 384) == 2 * 1 * 384
+    assert L.mbok_alpha_elems(3, 4096, 4096) == 4096 * 32 * 3
+    assert L.mbok_alpha_elems(2, 13, 256) == 16 * 2 * 2
+    assert L.mbok_packed_bytes(0, 8, 128) == 0
+    assert L.mbok_packed_bytes(1, 8, 100) == 0
+    assert L.mbok_gemv_workspace_bytes(3, 4096, 512, 1) == 0       # one slab: no workspace
+    assert L.mbok_gemv_workspace_bytes(3, 4096, 4096, 1) > 8 * 4096 * 4
+    assert L.mbok_gemv_workspace_bytes(3, 4096, 4096, 17) == 0
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.mbok_status_string(s).decode() not in ("", "unknown status")
+    assert L.mbok_status_string(99).decode() == "unknown status"
+
+
+def test_gemv_argument_errors(L):
+    g = lambda **kw: L.mbok_gemv(*[kw.get(k, v) for k, v in dict(
+        packed=FAKE, alpha=FAKE, K=3, M=64, N=1024, group=128, x=FAKE, dt=1, batch=1, y=FAKE,
+        ws=FAKE, wsb=1 << 20, stream=None).items()])
+    assert g(K=0) == 1 and g(K=5) == 1
+    assert g(M=0) == 2 and g(N=100) == 2 and g(N=0) == 2
+    assert g(group=64) == 4
+    assert g(packed=None) == 1 and g(x=None) == 1 and g(y=None) == 1
+    assert g(dt=7) == 1
+    assert g(batch=0) == 1 and g(batch=17) == 1
+    assert g(x=FAKE_ODD) == 3 and g(packed=FAKE + 4) == 3
+    assert g(ws=None) == 6 and g(wsb=16) == 6
+
+
+def test_gemm_and_pack_argument_errors(L):
+    assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 128, FAKE, 0, FAKE, None) == 2
+    assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 256, FAKE, 8, FAKE, None) == 4
+    assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 128, FAKE_ODD, 8, FAKE, None) == 3
+    assert L.mbok_gemm(None, FAKE, 3, 64, 256, 128, FAKE, 8, FAKE, None) == 1
+    assert L.mbok_pack_bits(None, 1, 8, 128, FAKE, None) == 1
+    assert L.mbok_pack_bits(FAKE, 1, 8, 130, FAKE, None) == 2
+    assert L.mbok_pack_bits(FAKE_ODD, 1, 8, 128, FAKE, None) == 3
+    assert L.mbok_pack_alpha(FAKE, 5, 8, 128, FAKE, None) == 1
+    assert L.mbok_residual_binarize(FAKE, 8, 128, 2, 64, FAKE, FAKE, None, None) == 4
+    assert L.mbok_residual_binarize(FAKE, 8, 128, 2, 128, FAKE, FAKE, FAKE_ODD, None) == 3
+    assert L.mbok_residual_binarize(FAKE, 0, 128, 2, 128, FAKE, FAKE, None, None) == 2
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    s = torch.ones(1, 8, 128, dtype=torch.int8)
+    with pytest.raises(ValueError):
+        mb.pack_bits(s, 1, 8, 128, torch.empty(64, dtype=torch.int32))

@@ -1,0 +1,234 @@
+"""GPU parity: every call of the C ABI against the CPU oracle on the same
+seeded inputs.  Packing, scale blocking and residual binarisation must match
+bit for bit; matrix products must meet the stated tolerance
+(|y - y_ref| <= 1e-3 * sum_j |W x| + 1e-6 per element; relative L2 <= 1e-5
+for the fp32-output GEMV)."""
+import numpy as np
+import pytest
+
+from oracle import mbok_oracle as O
+from boolean_weight_matmul_b200 import workloads as wl
+from helpers import (GEMV_REL_L2, alpha_blocked_gpu, assert_close, ensure_built, gemm_gpu,
+                     gemv_gpu, packed_from_signs_gpu, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    ensure_built()
+
+
+def _words_u32(t) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint32)
+
+
+# --------------------------------------------------------------------------
+# Packing
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,M,N", [(1, 1, 128), (3, 13, 384), (4, 129, 256), (2, 256, 512),
+                                   (3, 4096, 4096)])
+def test_pack_bits_bit_exact(K, M, N):
+    s = wl.random_signs(K, M, N, 200 + K + M, p_zero=0.05)
+    got = _words_u32(packed_from_signs_gpu(s))
+    assert np.array_equal(got, O.pack_signs(s))
+
+
+@pytest.mark.parametrize("K,M,N", [(1, 1, 128), (3, 13, 384), (4, 4096, 4096)])
+def test_pack_alpha_bit_exact(K, M, N):
+    a = wl.alpha_decaying(K, M, N, 300 + K)
+    got = alpha_blocked_gpu(a, K, M, N).cpu().numpy()
+    assert np.array_equal(got.view(np.uint16), O.block_alpha(a, K, M, N).view(np.uint16))
+
+
+# --------------------------------------------------------------------------
+# Residual binarisation (bit-exact)
+# --------------------------------------------------------------------------
+
+def _residual_gpu(W: np.ndarray, K: int):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    M, N = W.shape
+    Wd = to_dev(W)
+    packed = mb.empty_packed(K, M, N)
+    alpha = mb.empty_alpha(K, M, N)
+    R = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    mb.residual_binarize(Wd, M, N, K, 128, packed, alpha, R)
+    torch.cuda.synchronize()
+    return _words_u32(packed), alpha.cpu().numpy(), R.cpu().numpy()
+
+
+def _check_residual(W, K):
+    M, N = W.shape
+    pw, pa, pr = _residual_gpu(W, K)
+    s, a, R = O.residual_binarize(W, K)
+    assert np.array_equal(pw, O.pack_signs(s)), "packed kernels differ"
+    assert np.array_equal(pa.view(np.uint16), O.block_alpha(a, K, M, N).view(np.uint16)), "scales differ"
+    assert np.array_equal(pr.view(np.uint32), R.view(np.uint32)), "residual differs"
+
+
+@pytest.mark.parametrize("K,M,N", [(1, 256, 512), (3, 256, 512), (4, 13, 384), (2, 1, 128)])
+def test_residual_bit_exact_small(K, M, N):
+    _check_residual(wl.w_normal(M, N, wl.seed_of(1, K, 3)), K)
+
+
+def test_residual_edge_cases():
+    # zero and negative-zero groups (sign(0) = +1, alpha = 0), and a group whose
+    # mean sits just above an fp16 midpoint (single rounding from fp64).
+    W = wl.w_normal(9, 384, 77)
+    W[0, :128] = 0.0
+    W[1, 128:256] = -0.0
+    W[2, :] = 1.0
+    W[2, 5] = 1 + 2.0 ** -4
+    W[2, 77] = 1 + 2.0 ** -23
+    for K in (1, 3):
+        _check_residual(W, K)
+
+
+@pytest.mark.parametrize("K,M,N", [(3, 11008, 4096), (2, 4096, 11008)])
+def test_residual_bit_exact_llama7b_mlp(K, M, N):
+    _check_residual(wl.w_normal(M, N, wl.seed_of(3, 0 if M > N else 2, 3)), K)
+
+
+# --------------------------------------------------------------------------
+# Decode / small-batch GEMV
+# --------------------------------------------------------------------------
+
+def _gemv_case(K, M, N, batch, x_dtype, seed, alpha_kind="abs_normal", rows=None, p_zero=0.0):
+    s = wl.random_signs(K, M, N, seed, p_zero=p_zero)
+    a = (wl.alpha_abs_normal if alpha_kind == "abs_normal" else wl.alpha_decaying)(K, M, N, seed + 1)
+    x = wl.x_normal(batch, N, seed + 2, x_dtype)
+    y = gemv_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, x, x_dtype)
+    y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, x, x_dtype, rows=rows)
+    if rows is not None:
+        y = y[:, rows]
+    return y, y_ref, E
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+@pytest.mark.parametrize("M,N", [(1, 128), (7, 256), (13, 640), (128, 512), (129, 1024), (64, 1536)])
+def test_gemv_small_shapes(K, M, N):
+    for x_dtype in ("f32", "bf16"):
+        y, y_ref, E = _gemv_case(K, M, N, 1, x_dtype, 1000 + 17 * K + M + N)
+        assert_close(y, y_ref, E, GEMV_REL_L2, f"K={K} M={M} N={N} {x_dtype}")
+
+
+@pytest.mark.parametrize("batch", [2, 3, 4, 16])
+def test_gemv_small_batch(batch):
+    y, y_ref, E = _gemv_case(3, 200, 1152, batch, "bf16", 4000 + batch, "decaying")
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"batch={batch}")
+
+
+def test_gemv_toy_workload_f32():
+    w = wl.TOY_GEMV
+    s = wl.random_signs(w.K, w.M, w.N, wl.seed_of(1, 0, 4))
+    a = wl.alpha_abs_normal(w.K, w.M, w.N, wl.seed_of(1, 0, 1))
+    x = wl.x_normal(1, w.N, wl.seed_of(1, 0, 2), "f32")
+    y = gemv_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, w.K, w.M, w.N), w.K, w.M, w.N, x, "f32")
+    y_ref, E = O.linear(O.pack_signs(s), a, w.K, w.M, w.N, x, "f32")
+    assert_close(y, y_ref, E, GEMV_REL_L2, w.name)
+
+
+def test_gemv_q_proj_full_random_words():
+    # LLaMA-7B q_proj, K=3, batch 1, Bernoulli(0.5) words as drawn (layout-free),
+    # decaying scales; every output row checked.
+    import torch
+    w = wl.Q_PROJ_7B
+    K, M, N = w.K, w.M, w.N
+    words = wl.random_words(O.packed_bytes(K, M, N) // 4, wl.seed_of(2, 0, 0))
+    a = wl.alpha_decaying(K, M, N, wl.seed_of(2, 0, 1))
+    x = wl.x_normal(1, N, wl.seed_of(2, 0, 2))
+    packed = to_dev(words.view(np.int32))
+    y = gemv_gpu(packed, alpha_blocked_gpu(a, K, M, N), K, M, N, x, "bf16")
+    y_ref, E = O.linear(words, a, K, M, N, x, "bf16")
+    assert_close(y, y_ref, E, GEMV_REL_L2, w.name)
+    del packed
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("which,K,batch", [("gate", 3, 1), ("down", 2, 4), ("up", 3, 16)])
+def test_gemv_llama7b_mlp_residual_weights(which, K, batch):
+    # Weights from the GPU residual binarisation of W ~ N(0, 0.02^2) (the
+    # workload recipe); oracle on 384 sampled rows.
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    w = wl.mlp_7b(K, which, batch)
+    M, N = w.M, w.N
+    W = wl.w_normal(M, N, wl.seed_of(3, 1, 3))
+    packed = mb.empty_packed(K, M, N)
+    alpha = mb.empty_alpha(K, M, N)
+    mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
+    x = wl.x_normal(batch, N, wl.seed_of(3, 1, 2))
+    y = gemv_gpu(packed, alpha, K, M, N, x, "bf16")
+    words = _words_u32(packed)
+    a_mgk = O.unblock_alpha(alpha.cpu().numpy(), K, M, N)
+    rows = np.sort(np.random.default_rng(9).choice(M, 384, replace=False))
+    y_ref, E = O.linear(words, a_mgk, K, M, N, x, "bf16", rows=rows)
+    assert_close(y[:, rows], y_ref, E, GEMV_REL_L2, w.name)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,M,N", [("q", 5120, 5120), ("gate", 13824, 5120), ("down", 5120, 13824)])
+def test_gemv_llama13b_shapes_k4_sampled(name, M, N):
+    y, y_ref, E = _gemv_case(4, M, N, 1, "bf16", 5000 + M + N, "decaying",
+                             rows=np.sort(np.random.default_rng(M).choice(M, 256, replace=False)))
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"llama13b {name}")
+
+
+def test_gemv_flip_invariance_bitwise():
+    # Flipping every bit of kernel k and negating its scales gives the same y
+    # bit for bit (each lookup negates exactly).
+    K, M, N = 3, 300, 1536
+    s = wl.random_signs(K, M, N, 61)
+    a = wl.alpha_decaying(K, M, N, 62)
+    x = wl.x_normal(1, N, 63)
+    y0 = gemv_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, x, "bf16")
+    for k in range(K):
+        s2, a2 = s.copy(), a.copy()
+        s2[k] = -s2[k]
+        a2[:, :, k] = -a2[:, :, k]
+        y1 = gemv_gpu(packed_from_signs_gpu(s2), alpha_blocked_gpu(a2, K, M, N), K, M, N, x, "bf16")
+        assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
+
+
+def test_gemv_deterministic():
+    K, M, N = 3, 4096, 4096
+    s = wl.random_signs(K, M, N, 71)
+    a = wl.alpha_decaying(K, M, N, 72)
+    x = wl.x_normal(1, N, 73)
+    p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
+    y0 = gemv_gpu(p, al, K, M, N, x, "bf16")
+    y1 = gemv_gpu(p, al, K, M, N, x, "bf16")
+    assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# Prefill GEMM
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,M,N,T", [(1, 128, 128, 1), (3, 200, 384, 37), (4, 129, 512, 130),
+                                     (2, 64, 1024, 256)])
+def test_gemm_small(K, M, N, T):
+    s = wl.random_signs(K, M, N, 800 + T)
+    a = wl.alpha_decaying(K, M, N, 801 + T)
+    X = wl.x_normal(T, N, 802 + T)
+    Y = gemm_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, X)
+    Y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, X, "bf16")
+    assert_close(Y, Y_ref, E, None, f"gemm K={K} M={M} N={N} T={T}")
+
+
+def test_gemm_prefill_q_proj_sampled():
+    # LLaMA-7B q_proj prefill: K=3, 4096 x 4096, 2048 tokens; 128 sampled rows.
+    w = wl.PREFILL_7B
+    K, M, N, T = w.K, w.M, w.N, w.tokens
+    words = wl.random_words(O.packed_bytes(K, M, N) // 4, wl.seed_of(4, 0, 0))
+    a = wl.alpha_decaying(K, M, N, wl.seed_of(4, 0, 1))
+    X = wl.x_normal(T, N, wl.seed_of(4, 0, 2))
+    Y = gemm_gpu(to_dev(words.view(np.int32)), alpha_blocked_gpu(a, K, M, N), K, M, N, X)
+    rows = np.sort(np.random.default_rng(4).choice(M, 128, replace=False))
+    Y_ref, E = O.linear(words, a, K, M, N, X, "bf16", rows=rows)
+    assert_close(Y[:, rows], Y_ref, E, None, w.name)
