@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
             "mbok_residual_binarize": ([vp, i, i, i, i, vp, vp, vp, vp], i),
             "mbok_gemv": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp], i),
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
+            "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -150,6 +151,13 @@ def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=
                                             if isinstance(workspace, torch.Tensor) else 0)
     _check(lib().mbok_gemv(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype, batch,
                            _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv")
+
+
+def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=None) -> None:
+    """mbok_gemv for callers that cannot allocate: scratch comes from the
+    library's built-in array (see include/mbok.h)."""
+    _check(lib().mbok_gemv_noalloc(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype,
+                                   batch, _ptr(y), _stream(stream)), "mbok_gemv_noalloc")
 
 
 def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:

@@ -47,6 +47,7 @@ const char* mbok_status_string(int status) {
     case MBOK_ERR_UNSUPPORTED: return "unsupported option";
     case MBOK_ERR_CUDA: return "CUDA launch error";
     case MBOK_ERR_WORKSPACE: return "workspace missing or too small";
+    case MBOK_ERR_SCRATCH_LIMIT: return "problem exceeds the built-in scratch of mbok_gemv_noalloc";
     default: return "unknown status";
   }
 }

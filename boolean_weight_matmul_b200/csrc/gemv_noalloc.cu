@@ -1,0 +1,80 @@
+// mbok_gemv_noalloc: the decode GEMV for callers that cannot allocate device
+// memory.  Its scratch (the per-slab partial sums and arrival counters that
+// mbok_gemv keeps in a caller-provided workspace) lives in a fixed-size array
+// compiled into this library instead.  The library allocates nothing here.
+#include "mbok_common.cuh"
+
+namespace mbok {
+cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
+                            float*, void*, cudaStream_t);
+size_t gemv_lut_workspace_bytes(const Shape&);
+}  // namespace mbok
+
+using namespace mbok;
+
+// The scratch array.  Every GPU that loads the library holds it until the
+// process exits.  In host code `g_noalloc_scratch` names a host-side stand-in,
+// not the device array, so host code only ever passes the device address
+// obtained from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MBOK_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// The arrival counters occupy the first bytes of any GEMV workspace; they must
+// read zero when a call starts.
+constexpr size_t kCounterBytesToClear = 1024 * sizeof(unsigned);
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Set-up, once per device, with that device current: the device address of
+// the scratch array.  Returns nullptr if the runtime refuses.
+void* scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = ptr;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int M,
+                                 int N, int group, const void* x, int x_dtype, int batch, float* y,
+                                 void* stream) {
+  if (K < 1 || K > MBOK_MAX_K) return MBOK_ERR_INVALID_ARG;
+  if (M < 1 || N < MBOK_GROUP || N % MBOK_GROUP != 0 || M > (1 << 22) || N > (1 << 20))
+    return MBOK_ERR_SHAPE;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (packed == nullptr || alpha == nullptr || x == nullptr || y == nullptr)
+    return MBOK_ERR_INVALID_ARG;
+  if (x_dtype != MBOK_F32 && x_dtype != MBOK_BF16) return MBOK_ERR_INVALID_ARG;
+  if (batch < 1 || batch > MBOK_MAX_BATCH) return MBOK_ERR_INVALID_ARG;
+  const uintptr_t a16 = 15;
+  if ((reinterpret_cast<uintptr_t>(packed) & a16) || (reinterpret_cast<uintptr_t>(alpha) & a16) ||
+      (reinterpret_cast<uintptr_t>(x) & a16) || (reinterpret_cast<uintptr_t>(y) & 3))
+    return MBOK_ERR_ALIGN;
+  const Shape s = make_shape(K, M, N);
+  const size_t need = gemv_lut_workspace_bytes(s);
+  if (need > size_t(MBOK_NOALLOC_SCRATCH_BYTES)) return MBOK_ERR_SCRATCH_LIMIT;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  if (need > 0) {
+    scratch = scratch_address();
+    if (scratch == nullptr) return MBOK_ERR_CUDA;
+    // The array keeps whatever the previous call left: clear the counters.
+    if (cudaMemsetAsync(scratch, 0, kCounterBytesToClear, st) != cudaSuccess) return MBOK_ERR_CUDA;
+  }
+  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
+    if (launch_gemv_lut(reinterpret_cast<const uint8_t*>(packed), alpha, s, xb,
+                        x_dtype == MBOK_F32, y + size_t(b) * M, scratch, st) != cudaSuccess)
+      return MBOK_ERR_CUDA;
+  }
+  return MBOK_OK;
+}

@@ -52,7 +52,8 @@ typedef enum {
   MBOK_ERR_ALIGN = 3,         /* a pointer lacks its required alignment */
   MBOK_ERR_UNSUPPORTED = 4,   /* group != 128 */
   MBOK_ERR_CUDA = 5,          /* a kernel launch failed */
-  MBOK_ERR_WORKSPACE = 6      /* workspace NULL or smaller than required */
+  MBOK_ERR_WORKSPACE = 6,     /* workspace NULL or smaller than required */
+  MBOK_ERR_SCRATCH_LIMIT = 7  /* problem needs more than MBOK_NOALLOC_SCRATCH_BYTES */
 } mbok_status;
 
 typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
@@ -61,6 +62,8 @@ typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
 #define MBOK_LAYOUT_VERSION 1
 #define MBOK_MAX_K 4
 #define MBOK_MAX_BATCH 16
+/* Size of the scratch array built into the library for mbok_gemv_noalloc. */
+#define MBOK_NOALLOC_SCRATCH_BYTES (4u << 20)
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mbok_status_string(int status);
@@ -129,6 +132,33 @@ int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint3
 int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
               const void* x, int x_dtype, int batch, float* y, void* workspace,
               size_t workspace_bytes, void* stream);
+
+/* mbok_gemv without a workspace argument, for callers that cannot allocate
+ * device memory: code that must not call cudaMalloc after start-up (an
+ * allocator-free or real-time serving loop), code that runs where allocation
+ * is forbidden or would break the caller's memory accounting (a plugin inside
+ * a host framework that owns every device buffer), or a C caller with no
+ * allocator of its own.  (The method's pages have no counterpart; this is a
+ * property of the library, not of the method.)
+ *
+ * Same arguments, results and accuracy as mbok_gemv, minus the workspace.
+ * The scratch mbok_gemv would take from the workspace comes instead from one
+ * array of MBOK_NOALLOC_SCRATCH_BYTES (4 MiB) compiled into the library; every
+ * GPU that loads the library holds that array until the process exits.  This
+ * entry point calls no allocating routine (no cudaMalloc / cudaFree).
+ *  - Limit: shapes whose mbok_gemv_workspace_bytes exceeds
+ *    MBOK_NOALLOC_SCRATCH_BYTES are rejected with MBOK_ERR_SCRATCH_LIMIT
+ *    (roughly M * N > 500 million weights).
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    CUDA stream capture on that device.
+ *  - Each call first clears, on `stream`, the part of the array that must
+ *    start at zero; the rest keeps what the previous call left.
+ *  - All calls in the process share the one array: calls that may overlap on
+ *    the GPU (different streams without ordering, or several host threads)
+ *    race and give wrong results.  Order them on one stream. */
+int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N,
+                      int group, const void* x, int x_dtype, int batch, float* y, void* stream);
 
 /* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill), where Wt is W
  * rounded to bf16 element-wise, multiplied on the tensor cores with fp32

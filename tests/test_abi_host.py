@@ -57,7 +57,7 @@ def test_sizes(L):
 
 
 def test_status_strings(L):
-    for s in range(7):
+    for s in range(8):
         assert L.mbok_status_string(s).decode() not in ("", "unknown status")
     assert L.mbok_status_string(99).decode() == "unknown status"
 
