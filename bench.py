@@ -47,6 +47,8 @@ def args_parse():
     p.add_argument("--impl", choices=["mbok", "reference"], default="mbok")
     p.add_argument("--layers", type=int, default=48, help="distinct weight copies per step")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary rows")
+    p.add_argument("--rows", default="gemm,small_batch,sweep,residual,pack",
+                   help="comma-separated secondary rows to run")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -374,10 +376,22 @@ def run_gpu(a):
 def run_extras(torch, mb, wl, dev, peaks, a):
     """Secondary rows, each timed with CUDA events (graph replays)."""
     out = {}
+    rows = set(a.rows.split(","))
     stream = torch.cuda.Stream(device=dev)
     g = torch.Generator(device=dev)
     g.manual_seed(12345)
+    if "gemm" in rows:
+        run_gemm_row(torch, mb, wl, dev, peaks, stream, g, out)
+    if "small_batch" in rows:
+        run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out)
+    if "sweep" in rows:
+        run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out)
+    if "residual" in rows or "pack" in rows:
+        run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows)
+    return out
 
+
+def run_gemm_row(torch, mb, wl, dev, peaks, stream, g, out):
     # Prefill GEMM, K=3, 4096 x 4096, 2048 tokens.
     K, M, N, T = 3, 4096, 4096, 2048
     packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
@@ -392,10 +406,12 @@ def run_extras(torch, mb, wl, dev, peaks, a):
     tflops = 2.0 * M * N * T / (ms * 1e-3) / 1e12
     out["prefill_gemm_llama7b_q_proj_k3_t2048"] = {
         "us": 1e3 * ms, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-        "peak_tflops": peaks["bf16_tflops"], "kernel": "gemm_mma_kernel"}
+        "peak_tflops": peaks["bf16_tflops"], "kernel": "gemm_tc_kernel<3>"}
     del gr, packed, X, Y
     torch.cuda.empty_cache()
 
+
+def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
     # Small batch, LLaMA-7B gate 11008 x 4096, K=3 (and down 4096 x 11008, K=2).
     for (name, K, M, N) in (("gate", 3, 11008, 4096), ("down", 2, 4096, 11008)):
         L = 8
@@ -424,6 +440,8 @@ def run_extras(torch, mb, wl, dev, peaks, a):
         del packed, al
         torch.cuda.empty_cache()
 
+
+def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):
     # LLaMA-13B linear sweep, K=4, 40 layers x 7 matrices, batch 1.
     K = 4
     layers = wl.LLAMA13B_LAYERS
@@ -452,6 +470,8 @@ def run_extras(torch, mb, wl, dev, peaks, a):
     del gr, mats
     torch.cuda.empty_cache()
 
+
+def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
     # Residual binarisation, LLaMA-7B gate 11008 x 4096, K=3.
     K, M, N = 3, 11008, 4096
     W = torch.randn(M, N, device=dev, generator=g) * 0.02
@@ -467,7 +487,6 @@ def run_extras(torch, mb, wl, dev, peaks, a):
     ms, gr = time_graph(torch, lambda: mb.pack_bits(S, K, M, N, packed, stream=stream), 5, 2, stream)
     out["pack_bits_llama7b_gate_k3"] = {"ms": ms, "gbs_in": S.numel() / (ms * 1e-3) / 1e9}
     del gr
-    return out
 
 
 def main():

@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemv": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp], i),
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
+            "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -163,6 +164,13 @@ def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=Non
 def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:
     _check(lib().mbok_gemm(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(X), T, _ptr(Y),
                            _stream(stream)), "mbok_gemm")
+
+
+def read_device_errors() -> int:
+    """Flags of kernels whose bounded waits gave up since the last read (0 = none)."""
+    f = ctypes.c_uint(0)
+    _check(lib().mbok_read_device_errors(ctypes.byref(f)), "mbok_read_device_errors")
+    return f.value
 
 
 def dtype_code(x: torch.Tensor) -> int:

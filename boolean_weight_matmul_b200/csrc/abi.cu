@@ -11,8 +11,10 @@ cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __hal
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t);
 size_t gemv_lut_workspace_bytes(const Shape&);
-cudaError_t launch_gemm_mma(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
-                            uint16_t*, float*, cudaStream_t);
+unsigned gemv_error_flags();
+cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
+                           uint16_t*, cudaStream_t);
+unsigned gemm_error_flags();
 }  // namespace mbok
 
 using namespace mbok;
@@ -132,18 +134,28 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
   return MBOK_OK;
 }
 
+int mbok_read_device_errors(unsigned* flags) {
+  if (flags == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MBOK_ERR_CUDA;
+  const unsigned g = gemv_error_flags();
+  const unsigned m = gemm_error_flags();
+  if (g == ~0u || m == ~0u) return MBOK_ERR_CUDA;
+  *flags = (g ? 1u : 0u) | (m ? 2u : 0u);
+  return MBOK_OK;
+}
+
 int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
               const uint16_t* X, int T, uint16_t* Y, void* stream) {
   const int st = check_shape(K, M, N);
   if (st != MBOK_OK) return st;
   if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
-  if (T < 1 || T > (1 << 24)) return MBOK_ERR_SHAPE;
+  if (T < 1 || T > (1 << 23)) return MBOK_ERR_SHAPE;
   if (packed == nullptr || alpha == nullptr || X == nullptr || Y == nullptr)
     return MBOK_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(X, 16) || !aligned(Y, 16))
     return MBOK_ERR_ALIGN;
-  return from_cuda(launch_gemm_mma(reinterpret_cast<const uint8_t*>(packed), alpha,
-                                   make_shape(K, M, N), X, T, Y, nullptr, as_stream(stream)));
+  return from_cuda(launch_gemm_tc(reinterpret_cast<const uint8_t*>(packed), alpha, make_shape(K, M, N), X,
+                                  T, Y, as_stream(stream)));
 }
 
 }  // extern "C"

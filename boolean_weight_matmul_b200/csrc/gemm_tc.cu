@@ -1,0 +1,454 @@
+// Prefill GEMM  Y[t][r] = sum_j Wt[r][j] X[t][j]  on the sm_100a tensor cores
+// (tcgen05.mma, accumulator in tensor memory).
+//
+// W = sum_k alpha_k B_k (Paper-Notes page, 方法详解 / 关键设计: multi-kernel
+// Boolean weights with group-wise scales) is never stored densely: each CTA
+// unpacks the bf16 weight tile it needs into shared memory right before the
+// tensor cores read it.  Once decoded the product is a dense contraction, so
+// it runs as bf16 x bf16 -> fp32 MMAs.
+//
+// CTA tile: 128 weight rows (MMA M) x 256 tokens (MMA N), K-steps of 64
+// columns, a 4-stage shared-memory ring.  Per stage:
+//   * X tile, 256 tokens x 64 columns bf16 (32 KB): one TMA tensor load with
+//     128-byte swizzle (warp 0);
+//   * W tile, 128 rows x 64 columns bf16 (16 KB): written by 8 unpack warps in
+//     the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
+//     the two sign bits are brought to bit 15 and bit 31 by one shift of
+//     (h | h << 15), where h holds the row's 16 bits of one kernel, and
+//     applied to the bf16 scale pair with one LOP3; the K kernels are summed
+//     with packed bf16 adds (HADD2);
+//   * one thread (warp 1) issues 4 tcgen05.mma (M=128, N=256, K=16) into the
+//     tensor-memory accumulator and commits them to the stage's "empty"
+//     barrier.
+// The epilogue (4 warps, one per 32-lane quarter of tensor memory) reads the
+// accumulator with tcgen05.ld: TMEM lane = weight row, column = token, so a
+// warp's 32 lanes store 32 consecutive elements of one output row of Y.
+// Every mbarrier wait is bounded (1 s); on timeout the CTA records an error
+// flag, drains what it issued (bounded), frees its tensor memory and exits.
+#include <cuda.h>
+
+#include "mbok_common.cuh"
+
+namespace mbok {
+
+constexpr int kTcRows = 128;      // weight rows per CTA (MMA M)
+constexpr int kTcTokens = 256;    // tokens per CTA (MMA N)
+constexpr int kTcBK = 64;         // columns per stage (one 128-byte swizzle row)
+constexpr int kTcStages = 4;
+constexpr int kTcXBytes = kTcTokens * kTcBK * 2;   // 32 KB
+constexpr int kTcWBytes = kTcRows * kTcBK * 2;     // 16 KB
+constexpr int kTcStageBytes = kTcXBytes + kTcWBytes;
+constexpr int kTcUnpackWarps = 8;
+constexpr int kTcThreads = (2 + kTcUnpackWarps) * 32;          // TMA, MMA, 8 unpack
+constexpr int kTcSmem = kTcStages * kTcStageBytes + 1024 + 256;  // + alignment + barriers
+constexpr unsigned kTcTmemCols = 256;
+constexpr unsigned long long kTcWaitNs = 1000000000ull;
+constexpr unsigned long long kTcDrainNs = 200000000ull;
+
+// Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=256.
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTcTokens >> 3) << 17) |
+                              (uint32_t(kTcRows >> 4) << 24);
+
+__device__ unsigned int g_gemm_error;
+
+struct TcParams {
+  const uint8_t* packed;
+  const uint16_t* alpha;
+  uint16_t* Y;
+  Shape s;
+  int T;
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t tc_smem(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long tc_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void tc_mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc_smem(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void tc_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tc_smem(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tc_smem(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait for phase `parity`; false on timeout.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, unsigned parity, unsigned long long limit = kTcWaitNs) {
+  const uint32_t a = tc_smem(bar);
+  unsigned long long t0 = 0;
+  for (unsigned it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 255u) == 0) {
+      const unsigned long long t = tc_ns();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > limit) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tc_tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+          tc_smem(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(tc_smem(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (version 1 for sm_100).
+__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);        // start address
+  d |= uint64_t(1) << 16;                      // leading byte offset (unused for swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;              // stride byte offset
+  d |= uint64_t(1) << 46;                      // descriptor version
+  d |= uint64_t(2) << 61;                      // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(tc_smem(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Unpack: 2 rows x 16 columns of W (all K kernels) -> bf16 in the swizzled tile
+// ---------------------------------------------------------------------------
+
+// Sign-applied scale pair for columns (2i, 2i+1): the scale's sign flips
+// where the bit is 0 (-1).  u = h | (h << 15) holds bit b at b and at 15 + b,
+// so one left shift by 15 - 2i puts bit 2i at 15 and bit 2i+1 at 31.
+template <int I>
+__device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t a2) {
+  const uint32_t s = u << (15 - 2 * I);
+  uint32_t r;
+  // r = (~s & 0x80008000) ^ a2
+  asm("lop3.b32 %0, %1, %2, %3, 0xA6;\n" : "=r"(r) : "r"(s), "r"(0x80008000u), "r"(a2));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  __nv_bfloat162 z = __hadd2(x, y);
+  return *reinterpret_cast<uint32_t*>(&z);
+}
+
+template <int K>
+__device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_t a2[K], uint32_t out[8]) {
+  uint32_t u[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) u[k] = h[k] | (h[k] << 15);
+#define MBOK_PAIR(I)                                                     \
+  {                                                                      \
+    uint32_t v = tc_signed_pair<I>(u[0], a2[0]);                         \
+    _Pragma("unroll") for (int k = 1; k < K; ++k) v = bf16x2_add(v, tc_signed_pair<I>(u[k], a2[k])); \
+    out[I] = v;                                                          \
+  }
+  MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
+#undef MBOK_PAIR
+}
+
+// bf16 pair (a, a) from an fp16 scale.
+__device__ __forceinline__ uint32_t tc_scale_pair(uint32_t h16) {
+  const float a = __half2float(__ushort_as_half(uint16_t(h16)));
+  const __nv_bfloat16 b = __float2bfloat16_rn(a);
+  const uint32_t bb = __bfloat16_as_ushort(b);
+  return bb | (bb << 16);
+}
+
+template <int K>
+struct UnpackRegs {
+  uint32_t bits[K];    // rows 2j (low halfword) and 2j+1 (high halfword) of one unit
+  uint32_t alpha[K];   // scales of rows 2j, 2j+1 (fp16 pair)
+};
+
+// Thread mapping for unpack: 256 threads, thread -> (row pair rp = tid >> 2,
+// unit u = tid & 3) of the 128 x 64 tile: rows r0 + 2rp, +1; columns 16u..16u+15.
+template <int K>
+__device__ __forceinline__ void tc_load_unpack(const TcParams& p, int r0, int kb, int tid, UnpackRegs<K>& R) {
+  const int rp = tid >> 2, u = tid & 3;
+  const int r = r0 + 2 * rp;                 // even row; r and r+1 share an octet
+  const int o = r / kOctet, i = r % kOctet;
+  const int q = kb * (kTcBK / kUnit) + u;
+  const int g = q / kUnitsPerGroup;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    if (r < p.s.M) {
+      R.bits[k] = __ldg(reinterpret_cast<const uint32_t*>(p.packed + unit_offset(p.s, o, k, q) + 2 * i));
+      R.alpha[k] = __ldg(reinterpret_cast<const uint32_t*>(p.alpha + alpha_offset(p.s, o, g, k) + i));
+    } else {
+      R.bits[k] = 0;
+      R.alpha[k] = 0;
+    }
+  }
+}
+
+template <int K>
+__device__ __forceinline__ void tc_store_unpack(unsigned char* wtile, int tid, const UnpackRegs<K>& R) {
+  const int rp = tid >> 2, u = tid & 3;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int row = 2 * rp + half;
+    uint32_t h[K], a2[K], out[8];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      h[k] = half ? (R.bits[k] >> 16) : (R.bits[k] & 0xFFFFu);
+      a2[k] = tc_scale_pair(half ? (R.alpha[k] >> 16) : (R.alpha[k] & 0xFFFFu));
+    }
+    tc_unpack_row<K>(h, a2, out);
+    // 16 columns = chunks 2u and 2u+1 of the row's 128-byte line, swizzled
+    unsigned char* line = wtile + row * 128;
+    const int c0 = (2 * u) ^ (row & 7), c1 = (2 * u + 1) ^ (row & 7);
+    *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+
+template <int K>
+__global__ void __launch_bounds__(kTcThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
+  uint64_t* full_w = full_x + kTcStages;
+  uint64_t* empty = full_w + kTcStages;
+  uint64_t* done = empty + kTcStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * kTcRows;
+  const int t0 = blockIdx.y * kTcTokens;
+  const int nkb = p.s.N / kTcBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      tc_mbar_init(&full_x[s], 1);
+      tc_mbar_init(&full_w[s], kTcUnpackWarps * 32);
+      tc_mbar_init(&empty[s], 1);
+    }
+    tc_mbar_init(done, 1);
+    s_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(tc_smem(tmem_slot)),
+                 "r"(kTcTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---- TMA producer: X tiles ----
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % kTcStages;
+        if (kb >= kTcStages && !tc_wait(&empty[s], unsigned((kb / kTcStages) - 1) & 1u)) { ok = false; break; }
+        tc_arrive_expect_tx(&full_x[s], kTcXBytes);
+        tc_tma_load_2d(smem + s * kTcStageBytes, &xmap, kb * kTcBK, t0, &full_x[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % kTcStages;
+        const unsigned ph = unsigned(kb / kTcStages) & 1u;
+        if (!tc_wait(&full_x[s], ph) || !tc_wait(&full_w[s], ph)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t xs = tc_smem(smem + s * kTcStageBytes);
+        const uint32_t ws = xs + kTcXBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBK / 16; ++kk)
+          tc_mma(tmem, tc_desc_sw128(ws + kk * 32), tc_desc_sw128(xs + kk * 32), (kb > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      if (ok) tc_commit(done);
+    }
+  } else {
+    // ---- unpack warps ----
+    const int tid = threadIdx.x - 64;
+    UnpackRegs<K> cur, nxt;
+    tc_load_unpack<K>(p, r0, 0, tid, cur);
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kTcStages;
+      if (kb + 1 < nkb) tc_load_unpack<K>(p, r0, kb + 1, tid, nxt);
+      if (kb >= kTcStages && !tc_wait(&empty[s], unsigned((kb / kTcStages) - 1) & 1u)) { ok = false; break; }
+      tc_store_unpack<K>(smem + s * kTcStageBytes + kTcXBytes, tid, cur);
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
+      tc_arrive(&full_w[s]);
+      cur = nxt;
+    }
+  }
+
+  if (!ok) atomicOr(&s_fail, 1);
+  __syncthreads();
+  bool fail = s_fail != 0;
+
+  // ---- epilogue: warps 4..7 read TMEM quarter (warp & 3) ----
+  if (!fail && warp >= 4 && warp < 8) {
+    if (!tc_wait(done, 0)) {
+      atomicOr(&s_fail, 1);
+    } else {
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int r = r0 + 32 * quarter + lane;
+#pragma unroll 1
+      for (int c = 0; c < kTcTokens; c += 32) {
+        uint32_t v[32];
+        const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(c);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+              "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+              "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+              "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+        if (r < p.s.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = t0 + c + j;
+            if (t < p.T)
+              p.Y[size_t(t) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  fail = s_fail != 0;
+  if (fail && threadIdx.x == 0) {
+    // Record the failure and let every copy and MMA this CTA issued complete
+    // (bounded) before its shared memory and tensor memory are released.
+    atomicOr(&g_gemm_error, 1u);
+    for (int s = 0; s < kTcStages; ++s) {
+      (void)tc_wait(&full_x[s], 0u, kTcDrainNs);
+      (void)tc_wait(&full_x[s], 1u, kTcDrainNs);
+      (void)tc_wait(&empty[s], 0u, kTcDrainNs);
+      (void)tc_wait(&empty[s], 1u, kTcDrainNs);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTcTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+unsigned gemm_error_flags() {
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemm_error, sizeof(v)) != cudaSuccess) return ~0u;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(g_gemm_error, &zero, sizeof(zero)) != cudaSuccess) return ~0u;
+  return v;
+}
+
+template <int K>
+static cudaError_t launch_tc_k(const CUtensorMap& map, const TcParams& p, cudaStream_t stream) {
+  auto fn = gemm_tc_kernel<K>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((p.s.M + kTcRows - 1) / kTcRows, (p.T + kTcTokens - 1) / kTcTokens);
+  fn<<<grid, kTcThreads, kTcSmem, stream>>>(map, p);
+  return cudaGetLastError();
+}
+
+// Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
+cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const uint16_t* X,
+                           int T, uint16_t* Y, cudaStream_t stream) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(s.N), cuuint64_t(T)};
+  const cuuint64_t strides[1] = {cuuint64_t(s.N) * 2};
+  const cuuint32_t box[2] = {cuuint32_t(kTcBK), cuuint32_t(kTcTokens)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.packed = packed;
+  p.alpha = alpha;
+  p.Y = Y;
+  p.s = s;
+  p.T = T;
+  switch (s.K) {
+    case 1: return launch_tc_k<1>(map, p, stream);
+    case 2: return launch_tc_k<2>(map, p, stream);
+    case 3: return launch_tc_k<3>(map, p, stream);
+    default: return launch_tc_k<4>(map, p, stream);
+  }
+}
+
+}  // namespace mbok

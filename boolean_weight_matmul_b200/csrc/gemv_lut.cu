@@ -6,35 +6,58 @@
 // The prior-art operator on the FluxBin page (算子创新: LUT-based GEMV that
 // streams uint32 weight words, extracts pattern indices with bit operations
 // and fetches precomputed partial sums) motivates a lookup table; this kernel
-// is designed for the B200 shared-memory pipe instead:
+// is laid out for the B200 shared-memory pipe and HBM instead:
 //
 //  * Each lane owns 16 consecutive columns of a 512-column slab and keeps two
 //    256-entry fp32 tables in ITS OWN shared-memory bank: T_lo[e] (columns
 //    0..7 of its unit) and T_hi[e] (columns 8..15), T[e] = sum_i (e_i ? x : -x).
 //    Entry e of lane L sits at byte e*256 + 128*h + 4L, so every lookup of a
-//    warp touches 32 distinct banks: one wavefront per 8 weight bits.
-//  * One 16-byte load per lane brings 8 rows x 16 columns of one kernel
-//    (storage format 1), i.e. each warp load is 512 contiguous bytes.
-//  * Per (row, kernel) the lane adds two lookups and applies its group scale
-//    with one FMA (the lane's 16 columns lie in one group).
+//    warp touches 32 distinct banks: one wavefront per 8 weight bits.  The
+//    address of a lookup is one byte permute: (byte << 8) | 4L.
+//  * Each warp streams its own row octets (octet o_begin + warp + 8t) from HBM
+//    into a private 3-deep shared-memory ring with 16-byte cp.async copies:
+//    per (octet, kernel) one copy per lane (512 contiguous bytes per warp),
+//    plus the octet's 4 groups x K scale vectors.  The main loop has no
+//    block-wide barrier.  Launches use programmatic dependent launch: before
+//    waiting on the previous grid the kernel only prefetches its first octets
+//    into L2 (coherent, so safe even if the previous grid wrote the weights);
+//    the shared-memory copies, the read of x and every write happen after the
+//    wait.  A chain of layers thus overlaps one launch's tail with the next
+//    launch's HBM traffic.
+//  * Per (row pair, kernel) a lane does four lookups, one packed fp32x2 add
+//    and one packed fp32x2 FMA with the two rows' fp16 group scales.
 //  * The 32 lanes' partial sums of an octet's 8 rows are combined by a
-//    transposing butterfly (9 shuffles per lane per octet).
+//    transposing shuffle butterfly.
 //  * A CTA covers one slab and a contiguous range of row octets; slabs are
-//    combined deterministically: the last CTA of a row range to finish sums
-//    the per-slab partials in slab order.
+//    combined deterministically: the last CTA of a row range to arrive (one
+//    release/acquire atomic per CTA) sums the per-slab partials in slab order.
+//    (A thread-block-cluster reduction through distributed shared memory was
+//    measured slower here: its barriers wait for the slowest CTA.)
 // Tables are built exactly sign-symmetric (T[~e] == -T[e]), so flipping every
 // bit of a kernel and negating its scales reproduces y bit for bit.
 #include "mbok_common.cuh"
 
 namespace mbok {
 
-constexpr int kSlabCols = 512;                    // columns per slab (32 lanes x 16)
+constexpr int kSlabCols = 512;                  // columns per slab (32 lanes x 16)
+constexpr int kUnitsPerSlab = kSlabCols / kUnit;
+constexpr int kGroupsPerSlab = kSlabCols / kGroup;
 constexpr int kGemvThreads = 512;
 constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kLutBytes = 256 * 256;              // 256 entries x (32 lanes x 2 tables x 4 B)
-constexpr size_t kMaxCps = 1024;                  // max row ranges (counters) per call
+constexpr int kLutBytes = 256 * 256;            // 256 entries x (32 lanes x 2 tables x 4 B)
+constexpr size_t kMaxCps = 1024;                // max row ranges (counters) per call
 constexpr size_t kCounterBytes = kMaxCps * sizeof(unsigned);
-static_assert(kGemvWarps == 16, "table build assigns 16 warps to (table, 32-entry block)");
+constexpr int kDepth = 3;                       // octets in flight per warp
+constexpr int kPrefetchOctets = 16;             // L2 prefetch ahead of the dependency wait, per warp
+
+template <int K>
+struct StageGeom {
+  static constexpr int kBits = K * kUnitsPerSlab * 16;        // [k][lane][16 B]
+  static constexpr int kAlpha = kGroupsPerSlab * K * 16;      // [group][k][8 x fp16]
+  static constexpr int kBytes = kBits + kAlpha;               // one octet of one warp
+  static constexpr int kRing = kGemvWarps * kDepth * kBytes;
+  static constexpr int kSmem = kLutBytes + kRing;
+};
 
 struct GemvParams {
   const uint8_t* packed;
@@ -47,24 +70,87 @@ struct GemvParams {
   int nslab, cps;
 };
 
-template <int K>
-struct OctetRegs {
-  uint4 bits[K];
-  uint4 alpha[K];
-};
+// ---------------------------------------------------------------------------
+// PTX helpers: async copies, L2 prefetch, grid dependency control
+// ---------------------------------------------------------------------------
 
-template <int K>
-__device__ __forceinline__ void load_octet(const GemvParams& p, int o, int q, bool lane_ok,
-                                           OctetRegs<K>& r) {
-  const int g = q / kUnitsPerGroup;
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
+}
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// ---------------------------------------------------------------------------
+// Lookup tables
+// ---------------------------------------------------------------------------
+
+// sum_{i<4} (n_i ? v_i : -v_i), associated as ((v0 + v1) + v2) + v3 so that
+// complementing n negates the result exactly.
+__device__ __forceinline__ float signed_sum4(const float v[4], uint32_t n) {
+  float t = ((n & 1) ? v[0] : -v[0]) + ((n & 2) ? v[1] : -v[1]);
+  t = t + ((n & 4) ? v[2] : -v[2]);
+  return t + ((n & 8) ? v[3] : -v[3]);
+}
+
+// The 8 activations x[col0 .. col0+7] as fp32 (0 when !ok).
+template <bool XF32>
+__device__ __forceinline__ void load_x8(const void* x, int col0, bool ok, float v[8]) {
+  if (!ok) {
 #pragma unroll
-  for (int k = 0; k < K; ++k) {
-    if (lane_ok) {
-      r.bits[k] = __ldg(reinterpret_cast<const uint4*>(p.packed + unit_offset(p.s, o, k, q)));
-      r.alpha[k] = __ldg(reinterpret_cast<const uint4*>(p.alpha + alpha_offset(p.s, o, g, k)));
-    } else {
-      r.bits[k] = make_uint4(0, 0, 0, 0);
-      r.alpha[k] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    return;
+  }
+  if (XF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + col0);
+    const float4 t0 = p[0], t1 = p[1];
+    v[0] = t0.x; v[1] = t0.y; v[2] = t0.z; v[3] = t0.w;
+    v[4] = t1.x; v[5] = t1.y; v[6] = t1.z; v[7] = t1.w;
+  } else {
+    const uint4 t = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + col0);
+    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = bf16_bits_to_float(w[e] & 0xFFFFu);
+      v[2 * e + 1] = bf16_bits_to_float(w[e] >> 16);
+    }
+  }
+}
+
+// Warp w fills entries [32*(w&7), 32*(w&7)+32) of table h = w>>3 for all 32
+// lanes from that table's 8 activations c[]: T[e] = A[e & 15] + B[e >> 4],
+// A/B the signed sums of the table's low and high four columns.
+__device__ __forceinline__ void build_tables(unsigned char* tab, const float c[8], int warp, int lane) {
+  static_assert(kGemvWarps == 16, "the table build assigns 16 warps to (table, 32-entry block)");
+  const int h = warp >> 3, blk = warp & 7;
+  float A[16];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) A[n] = signed_sum4(c, uint32_t(n));
+  unsigned char* dst = tab + 128 * h + 4 * lane;
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const float B = signed_sum4(c + 4, uint32_t(2 * blk + m));
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      const int e = 32 * blk + 16 * m + n;
+      *reinterpret_cast<float*>(dst + size_t(e) * 256) = A[n] + B;
     }
   }
 }
@@ -73,30 +159,35 @@ __device__ __forceinline__ float lut(const unsigned char* base, uint32_t off) {
   return *reinterpret_cast<const float*>(base + off);
 }
 
+// One octet (8 rows x this lane's 16 columns) of K kernels from a stage.
 template <int K>
 __device__ __forceinline__ void octet_dot(const unsigned char* tab, uint32_t lane4,
-                                          const OctetRegs<K>& r, float acc[8]) {
+                                          const uint4* bits, const uint4* alpha, float2 acc[4]) {
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const uint32_t w[4] = {r.bits[k].x, r.bits[k].y, r.bits[k].z, r.bits[k].w};
-    const uint32_t a[4] = {r.alpha[k].x, r.alpha[k].y, r.alpha[k].z, r.alpha[k].w};
+    const uint4 wv = bits[k * kUnitsPerSlab];
+    const uint4 av = alpha[k];
+    const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+    const uint32_t a[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      // word i holds row 2i (low halfword) and row 2i+1 (high halfword)
-      const float t0 = lut(tab, ((w[i] << 8) & 0xFF00u) | lane4);          // row 2i,   cols 0..7
-      const float t1 = lut(tab + 128, (w[i] & 0xFF00u) | lane4);           // row 2i,   cols 8..15
-      const float t2 = lut(tab, ((w[i] >> 8) & 0xFF00u) | lane4);          // row 2i+1, cols 0..7
-      const float t3 = lut(tab + 128, ((w[i] >> 16) & 0xFF00u) | lane4);   // row 2i+1, cols 8..15
-      const float2 al = half2_bits_to_float2(a[i]);                       // scales of rows 2i, 2i+1
-      acc[2 * i] = fmaf(al.x, t0 + t1, acc[2 * i]);
-      acc[2 * i + 1] = fmaf(al.y, t2 + t3, acc[2 * i + 1]);
+      // word i holds row 2i (bytes 0,1) and row 2i+1 (bytes 2,3); byte b of the
+      // word indexes the table for its 8 columns at offset (byte << 8) | 4L.
+      const float t0 = lut(tab, __byte_perm(w[i], lane4, 0x5504));         // row 2i,   cols 0..7
+      const float t1 = lut(tab + 128, __byte_perm(w[i], lane4, 0x5514));   // row 2i,   cols 8..15
+      const float t2 = lut(tab, __byte_perm(w[i], lane4, 0x5524));         // row 2i+1, cols 0..7
+      const float t3 = lut(tab + 128, __byte_perm(w[i], lane4, 0x5534));   // row 2i+1, cols 8..15
+      const float2 s = __fadd2_rn(make_float2(t0, t2), make_float2(t1, t3));
+      acc[i] = __ffma2_rn(half2_bits_to_float2(a[i]), s, acc[i]);
     }
   }
 }
 
-// Sum acc[0..7] over the 32 lanes; returns, in every lane, the total of row
+// Sum acc (8 rows) over the 32 lanes; returns, in every lane, the total of row
 // ((lane >> 2) & 7).  Fixed order, hence deterministic.
-__device__ __forceinline__ float octet_reduce(const float acc[8], int lane) {
+__device__ __forceinline__ float octet_reduce(const float2 acc2[4], int lane) {
+  const float acc[8] = {acc2[0].x, acc2[0].y, acc2[1].x, acc2[1].y,
+                        acc2[2].x, acc2[2].y, acc2[3].x, acc2[3].y};
   const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
   float r1[4];
 #pragma unroll
@@ -120,112 +211,121 @@ __device__ __forceinline__ float octet_reduce(const float acc[8], int lane) {
   return r3;
 }
 
-// sum_{i<4} (n_i ? v_i : -v_i), associated as ((v0 + v1) + v2) + v3 so that
-// complementing n negates the result exactly.
-__device__ __forceinline__ float signed_sum4(const float v[4], uint32_t n) {
-  float t = ((n & 1) ? v[0] : -v[0]) + ((n & 2) ? v[1] : -v[1]);
-  t = t + ((n & 4) ? v[2] : -v[2]);
-  return t + ((n & 8) ? v[3] : -v[3]);
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+
+// Copy octet o (this warp's K x 512 columns of bits and its 4 groups x K
+// scale vectors) into stage `st`; one commit group per octet.
+template <int K>
+__device__ __forceinline__ void issue_octet(const GemvParams& p, int slab, int units, int groups, int o,
+                                            unsigned char* st, int lane) {
+  using G = StageGeom<K>;
+  if (lane < units) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      cp_async16(st + k * kUnitsPerSlab * 16 + lane * 16,
+                 p.packed + unit_offset(p.s, o, k, slab * kUnitsPerSlab + lane));
+  }
+  if (lane < groups * K)
+    cp_async16(st + G::kBits + lane * 16, p.alpha + alpha_offset(p.s, o, slab * kGroupsPerSlab, 0) + lane * 8);
+  cp_async_commit();
 }
 
-// The 8 activations x[col0 .. col0+7] as fp32 (0 when !ok).
-template <bool XF32>
-__device__ __forceinline__ void load_x8(const void* x, int col0, bool ok, float v[8]) {
-  if (!ok) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.f;
-    return;
-  }
-  if (XF32) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + col0);
-    const float4 t0 = __ldg(p), t1 = __ldg(p + 1);
-    v[0] = t0.x; v[1] = t0.y; v[2] = t0.z; v[3] = t0.w;
-    v[4] = t1.x; v[5] = t1.y; v[6] = t1.z; v[7] = t1.w;
-  } else {
-    const uint4 t = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + col0));
-    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[2 * e] = bf16_bits_to_float(w[e] & 0xFFFFu);
-      v[2 * e + 1] = bf16_bits_to_float(w[e] >> 16);
-    }
-  }
-}
-
-// Warp w fills entries [32*(w&7), 32*(w&7)+32) of table h = w>>3 for all 32
-// lanes: T[e] = A[e & 15] + B[e >> 4], A/B the signed sums of the table's low
-// and high four columns.
-template <bool XF32>
-__device__ __forceinline__ void build_tables(unsigned char* tab, const void* x, int col0, bool ok,
-                                             int warp, int lane) {
-  const int h = warp >> 3, blk = warp & 7;
-  float c[8];
-  load_x8<XF32>(x, col0 + 8 * h, ok, c);
-  float A[16];
-#pragma unroll
-  for (int n = 0; n < 16; ++n) A[n] = signed_sum4(c, uint32_t(n));
-  const float B0 = signed_sum4(c + 4, uint32_t(2 * blk));
-  const float B1 = signed_sum4(c + 4, uint32_t(2 * blk + 1));
-  unsigned char* dst = tab + 128 * h + 4 * lane;
-#pragma unroll
-  for (int n = 0; n < 32; ++n) {
-    const int e = 32 * blk + n;
-    *reinterpret_cast<float*>(dst + size_t(e) * 256) = A[n & 15] + ((n < 16) ? B0 : B1);
+template <int K>
+__device__ __forceinline__ void prefetch_octet(const GemvParams& p, int slab, int units, int groups, int o,
+                                               int lane) {
+  // 128-byte lines: units*16 bytes per kernel, groups*K*16 bytes of scales
+  if (lane < (units + 7) / 8 * K) {
+    const int k = lane / ((units + 7) / 8), l = lane % ((units + 7) / 8);
+    prefetch_l2(p.packed + unit_offset(p.s, o, k, slab * kUnitsPerSlab) + 128 * l);
+  } else if (lane < (units + 7) / 8 * K + (groups * K * 16 + 127) / 128) {
+    const int l = lane - (units + 7) / 8 * K;
+    prefetch_l2(reinterpret_cast<const uint8_t*>(p.alpha + alpha_offset(p.s, o, slab * kGroupsPerSlab, 0)) + 128 * l);
   }
 }
 
 template <int K, bool XF32>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p) {
-  extern __shared__ __align__(1024) unsigned char tab[];
-  __shared__ int s_last;
+  using G = StageGeom<K>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* tab = smem;
+  __shared__ int s_flag;
+
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int slab = blockIdx.x % p.nslab, c = blockIdx.x / p.nslab;
   const int o_begin = int((long long)c * p.s.O / p.cps);
   const int o_end = int((long long)(c + 1) * p.s.O / p.cps);
-  const int q = slab * 32 + lane;
-  const bool lane_ok = q < p.s.Q;
+  const int units = min(kUnitsPerSlab, p.s.Q - slab * kUnitsPerSlab);
+  const int groups = units / kUnitsPerGroup;
+  const int q = slab * kUnitsPerSlab + lane;
+  const bool lane_ok = lane < units;
   const uint32_t lane4 = 4u * lane;
   const int Mpad = p.s.O * kOctet;
+  unsigned char* ring = smem + kLutBytes + warp * kDepth * G::kBytes;
+  // this warp's octets: o_begin + warp + 8t, t = 0 .. n_mine-1
+  const int first = o_begin + warp;
+  const int n_mine = first < o_end ? (o_end - first + kGemvWarps - 1) / kGemvWarps : 0;
 
-  // Issue the first octet's loads before building the tables.
-  int o = o_begin + warp;
-  OctetRegs<K> cur;
-  if (o < o_end) load_octet<K>(p, o, q, lane_ok, cur);
+  // Before the dependency wait: only L2 prefetches of this warp's first octets.
+  for (int t = 0; t < kPrefetchOctets && t < n_mine; ++t)
+    prefetch_octet<K>(p, slab, units, groups, first + t * kGemvWarps, lane);
+  allow_dependents();
+  // Inputs and workspace may be written by the previous grid: wait for it.
+  grid_dependency_wait();
 
-  build_tables<XF32>(tab, p.x, q * kUnit, lane_ok, warp, lane);
+  // x first: its load must not queue behind this warp's weight copies.
+  float xv[8];
+  load_x8<XF32>(p.x, q * kUnit + 8 * (warp >> 3), lane_ok, xv);
+#pragma unroll
+  for (int t = 0; t < kDepth; ++t) {
+    if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
+    else cp_async_commit();   // keep one group per slot
+  }
+  build_tables(tab, xv, warp, lane);
   __syncthreads();
 
-  for (; o < o_end; o += kGemvWarps) {
-    OctetRegs<K> nxt;
-    const int on = o + kGemvWarps;
-    if (on < o_end) load_octet<K>(p, on, q, lane_ok, nxt);
-    float acc[8];
+  for (int t = 0; t < n_mine; ++t) {
+    unsigned char* st = ring + (t % kDepth) * G::kBytes;
+    cp_async_wait<kDepth - 1>();   // octet t has landed (this lane's copies)
+    __syncwarp();                  // ... and every lane's copies
+    float2 acc[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    octet_dot<K>(tab, lane4, cur, acc);
+    for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+    if (lane_ok) {
+      const uint4* bits = reinterpret_cast<const uint4*>(st) + lane;
+      const uint4* al = reinterpret_cast<const uint4*>(st + G::kBits) + (lane / kUnitsPerGroup) * K;
+      octet_dot<K>(tab, lane4, bits, al, acc);
+    }
+    __syncwarp();                  // all lanes are done reading the slot
+    if (t + kDepth < n_mine)
+      issue_octet<K>(p, slab, units, groups, first + (t + kDepth) * kGemvWarps, st, lane);
+    else
+      cp_async_commit();
     const float total = octet_reduce(acc, lane);
+    const int o = first + t * kGemvWarps;
     const int row = o * kOctet + ((lane >> 2) & 7);
     if ((lane & 3) == 0) {
       if (p.nslab == 1) {
         if (row < p.s.M) p.y[row] = total;
       } else {
-        p.partial[size_t(slab) * Mpad + row] = total;
+        __stcg(p.partial + size_t(slab) * Mpad + row, total);
       }
     }
-    cur = nxt;
   }
-
+  cp_async_wait<0>();
   if (p.nslab == 1) return;
-  __threadfence();
+
+  // Cross-slab combination: one release/acquire arrival per CTA; the last
+  // CTA of the row range adds the slabs' partials in slab order.
   __syncthreads();
   if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(&p.counter[c], 1u);
-    s_last = (prev == unsigned(p.nslab - 1));
-    if (s_last) p.counter[c] = 0u;  // every slab of this row range has arrived
+    const unsigned prev = atomic_add_acq_rel(&p.counter[c], 1u);
+    s_flag = (prev == unsigned(p.nslab - 1));
+    if (s_flag) p.counter[c] = 0u;  // every slab of this row range has arrived
   }
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (!s_flag) return;
   const int r_end = min(o_end * kOctet, p.s.M);
   for (int r = o_begin * kOctet + threadIdx.x; r < r_end; r += blockDim.x) {
     float sum = 0.f;
@@ -233,6 +333,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
     p.y[r] = sum;
   }
 }
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
 
 struct GemvPlan {
   int nslab, cps;
@@ -253,23 +357,40 @@ inline GemvPlan gemv_plan(const Shape& s, int sm_count) {
 // (at most kMaxCps ranges); calls leave them at zero.  Per-slab partial sums
 // follow.  The counter block has a fixed size so that calls of any shape can
 // share one workspace.
-
 size_t gemv_lut_workspace_bytes(const Shape& s) {
   const size_t nslab = (s.N + kSlabCols - 1) / kSlabCols;
   if (nslab <= 1) return 0;
   return kCounterBytes + nslab * size_t(s.O) * kOctet * sizeof(float);
 }
 
+// This kernel has no spin-waits (cp.async groups complete by themselves), so
+// it never records a device error flag.
+unsigned gemv_error_flags() { return 0u; }
+
 template <int K, bool XF32>
 static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) {
+  using G = StageGeom<K>;
   auto fn = gemv_lut8_kernel<K, XF32>;
   static bool attr_set = false;   // set once, outside any stream capture
   if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  fn<<<grid, kGemvThreads, kLutBytes, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = G::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -160,11 +160,23 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
 int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N,
                       int group, const void* x, int x_dtype, int batch, float* y, void* stream);
 
-/* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill), where Wt is W
- * rounded to bf16 element-wise, multiplied on the tensor cores with fp32
- * accumulation, and Y is rounded to bf16.  X: bf16 [T][N]; Y: bf16 [T][M];
- * both 16-byte aligned.  Accuracy: |Y - Y_exact| <= 1e-3 * sum_j |W x| + 1e-6
- * per element (bf16 weight and output rounding). */
+/* Diagnostic: waits inside the library's kernels are bounded (about a second);
+ * a kernel that gives up records a flag and returns early instead of hanging.
+ * Writes the flags accumulated on the current device since the last call to
+ * *flags (0 = none; bit 0 = a decode-GEMV copy never completed; bit 1 = a
+ * prefill-GEMM pipeline wait gave up) and clears them.  Synchronises the
+ * device.  Returns MBOK_ERR_CUDA if the flags cannot be read. */
+int mbok_read_device_errors(unsigned* flags);
+
+/* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill) on the tensor cores
+ * (tcgen05, fp32 accumulation in tensor memory).  Wt is W in bf16: each fp16
+ * scale is rounded to bf16 and the K signed scales of an element are summed
+ * in bf16 while the tile is unpacked into shared memory.  Y is rounded to
+ * bf16.  X: bf16 [T][N]; Y: bf16 [T][M]; both 16-byte aligned; 1 <= T <= 2^23.
+ * Accuracy: |Y - Y_exact| <= 1e-3 * sum_j |W x| + 2^-8 * |Y_exact| + 1e-6 per
+ * element (bf16 weights; the second term covers the bf16 rounding of Y
+ * itself).  Waits inside the kernel are bounded: see
+ * mbok_read_device_errors. */
 int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
               const uint16_t* X, int T, uint16_t* Y, void* stream);
 

@@ -77,6 +77,7 @@ def test_gemv_argument_errors(L):
 
 
 def test_gemm_and_pack_argument_errors(L):
+    assert L.mbok_read_device_errors(None) == 1
     assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 128, FAKE, 0, FAKE, None) == 2
     assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 256, FAKE, 8, FAKE, None) == 4
     assert L.mbok_gemm(FAKE, FAKE, 3, 64, 256, 128, FAKE_ODD, 8, FAKE, None) == 3
