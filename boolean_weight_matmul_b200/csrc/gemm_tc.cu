@@ -10,9 +10,10 @@
 // CTA tile: 128 weight rows (MMA M) x 256 tokens (MMA N), K-steps of 64
 // columns, a 4-stage shared-memory ring.  Per stage:
 //   * X tile, 256 tokens x 64 columns bf16 (32 KB): one TMA tensor load with
-//     128-byte swizzle (warp 0);
-//   * W tile, 128 rows x 64 columns bf16 (16 KB): written by 8 unpack warps in
-//     the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
+//     128-byte swizzle; the tile's packed bits (16 octets x K x 64 bytes) and
+//     scales (16 octets x K x 8 fp16) come with two more TMA loads (warp 0);
+//   * W tile, 128 rows x 64 columns bf16 (16 KB): written by 16 unpack warps
+//     (one row x 16 columns per thread) in the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
 //     the two sign bits are brought to bit 15 and bit 31 by one shift of
 //     (h | h << 15), where h holds the row's 16 bits of one kernel, and
 //     applied to the bf16 scale pair with one LOP3; the K kernels are summed
@@ -32,22 +33,27 @@
 namespace mbok {
 
 constexpr int kTcRows = 128;      // weight rows per CTA (MMA M)
-constexpr int kTcTokens = 256;    // tokens per CTA (MMA N)
+constexpr int kTcTokens = 256;    // largest token tile per CTA (MMA N); the host picks <= this
 constexpr int kTcBK = 64;         // columns per stage (one 128-byte swizzle row)
 constexpr int kTcStages = 4;
 constexpr int kTcXBytes = kTcTokens * kTcBK * 2;   // 32 KB
 constexpr int kTcWBytes = kTcRows * kTcBK * 2;     // 16 KB
-constexpr int kTcStageBytes = kTcXBytes + kTcWBytes;
-constexpr int kTcUnpackWarps = 8;
-constexpr int kTcThreads = (2 + kTcUnpackWarps) * 32;          // TMA, MMA, 8 unpack
+constexpr int kTcOctets = kTcRows / kOctet;        // 16 row octets per tile
+constexpr int kTcBitsRow = kTcBK / 8;              // 64 columns = 8 bytes per row = 64 bytes per octet
+constexpr int kTcBitsBytes = kTcOctets * MBOK_MAX_K * kTcBitsRow * kOctet;   // 4 KB (K = 4)
+constexpr int kTcAlphaBytes = kTcOctets * MBOK_MAX_K * 16;                 // 1 KB (K = 4)
+constexpr int kTcStageBytes = kTcXBytes + kTcWBytes + kTcBitsBytes + kTcAlphaBytes;
+constexpr int kTcUnpackWarps = 16;
+constexpr int kTcThreads = (2 + kTcUnpackWarps) * 32;          // TMA, MMA, 16 unpack
 constexpr int kTcSmem = kTcStages * kTcStageBytes + 1024 + 256;  // + alignment + barriers
 constexpr unsigned kTcTmemCols = 256;
 constexpr unsigned long long kTcWaitNs = 1000000000ull;
 constexpr unsigned long long kTcDrainNs = 200000000ull;
 
-// Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=256.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTcTokens >> 3) << 17) |
-                              (uint32_t(kTcRows >> 4) << 24);
+// Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=n.
+inline uint32_t tc_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTcRows >> 4) << 24);
+}
 
 __device__ unsigned int g_gemm_error;
 
@@ -57,6 +63,8 @@ struct TcParams {
   uint16_t* Y;
   Shape s;
   int T;
+  int n_tile;       // tokens per CTA tile (multiple of 16, <= kTcTokens)
+  uint32_t idesc;   // instruction descriptor for N = n_tile
 };
 
 // ---------------------------------------------------------------------------
@@ -126,12 +134,13 @@ __device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
   const uint32_t z = 0;
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
 }
 
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -188,52 +197,28 @@ __device__ __forceinline__ uint32_t tc_scale_pair(uint32_t h16) {
   return bb | (bb << 16);
 }
 
+// Unpack one row x 16 columns: thread tid -> row r = tid >> 2, unit u = tid & 3
+// of the 128 x 64 tile.  Bits and scales come from the stage's TMA-loaded
+// copies: bits [octet][k][unit][row] halfwords, scales [octet][k][row] fp16.
 template <int K>
-struct UnpackRegs {
-  uint32_t bits[K];    // rows 2j (low halfword) and 2j+1 (high halfword) of one unit
-  uint32_t alpha[K];   // scales of rows 2j, 2j+1 (fp16 pair)
-};
-
-// Thread mapping for unpack: 256 threads, thread -> (row pair rp = tid >> 2,
-// unit u = tid & 3) of the 128 x 64 tile: rows r0 + 2rp, +1; columns 16u..16u+15.
-template <int K>
-__device__ __forceinline__ void tc_load_unpack(const TcParams& p, int r0, int kb, int tid, UnpackRegs<K>& R) {
-  const int rp = tid >> 2, u = tid & 3;
-  const int r = r0 + 2 * rp;                 // even row; r and r+1 share an octet
-  const int o = r / kOctet, i = r % kOctet;
-  const int q = kb * (kTcBK / kUnit) + u;
-  const int g = q / kUnitsPerGroup;
+__device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, const unsigned char* alpha,
+                                                    unsigned char* wtile, int tid) {
+  const int r = tid >> 2, u = tid & 3;
+  const int o = r >> 3, i = r & 7;
+  uint32_t h[K], a2[K], out[8];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    if (r < p.s.M) {
-      R.bits[k] = __ldg(reinterpret_cast<const uint32_t*>(p.packed + unit_offset(p.s, o, k, q) + 2 * i));
-      R.alpha[k] = __ldg(reinterpret_cast<const uint32_t*>(p.alpha + alpha_offset(p.s, o, g, k) + i));
-    } else {
-      R.bits[k] = 0;
-      R.alpha[k] = 0;
-    }
+    h[k] = *reinterpret_cast<const uint16_t*>(bits + ((o * K + k) * 4 + u) * 16 + 2 * i);
+    a2[k] = tc_scale_pair(*reinterpret_cast<const uint16_t*>(alpha + (o * K + k) * 16 + 2 * i));
   }
-}
-
-template <int K>
-__device__ __forceinline__ void tc_store_unpack(unsigned char* wtile, int tid, const UnpackRegs<K>& R) {
-  const int rp = tid >> 2, u = tid & 3;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int row = 2 * rp + half;
-    uint32_t h[K], a2[K], out[8];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      h[k] = half ? (R.bits[k] >> 16) : (R.bits[k] & 0xFFFFu);
-      a2[k] = tc_scale_pair(half ? (R.alpha[k] >> 16) : (R.alpha[k] & 0xFFFFu));
-    }
-    tc_unpack_row<K>(h, a2, out);
-    // 16 columns = chunks 2u and 2u+1 of the row's 128-byte line, swizzled
-    unsigned char* line = wtile + row * 128;
-    const int c0 = (2 * u) ^ (row & 7), c1 = (2 * u + 1) ^ (row & 7);
-    *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
-    *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
-  }
+  tc_unpack_row<K>(h, a2, out);
+  // 16 columns = chunks 2u and 2u+1 of the row's 128-byte line, swizzled; the
+  // 8 threads of a store phase hold 2 rows of opposite parity x 4 units, i.e.
+  // 8 distinct chunks.
+  unsigned char* line = wtile + r * 128;
+  const int c0 = (2 * u) ^ (r & 7), c1 = (2 * u + 1) ^ (r & 7);
+  *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
 // ---------------------------------------------------------------------------
@@ -242,10 +227,11 @@ __device__ __forceinline__ void tc_store_unpack(unsigned char* wtile, int tid, c
 
 template <int K>
 __global__ void __launch_bounds__(kTcThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
+               const __grid_constant__ CUtensorMap amap, TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
+  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // TMA data landed
   uint64_t* full_w = full_x + kTcStages;
   uint64_t* empty = full_w + kTcStages;
   uint64_t* done = empty + kTcStages;
@@ -254,7 +240,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = blockIdx.x * kTcRows;
-  const int t0 = blockIdx.y * kTcTokens;
+  const int t0 = blockIdx.y * p.n_tile;
   const int nkb = p.s.N / kTcBK;
 
   if (threadIdx.x == 0) {
@@ -285,8 +271,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
       for (int kb = 0; kb < nkb && ok; ++kb) {
         const int s = kb % kTcStages;
         if (kb >= kTcStages && !tc_wait(&empty[s], unsigned((kb / kTcStages) - 1) & 1u)) { ok = false; break; }
-        tc_arrive_expect_tx(&full_x[s], kTcXBytes);
-        tc_tma_load_2d(smem + s * kTcStageBytes, &xmap, kb * kTcBK, t0, &full_x[s]);
+        unsigned char* st = smem + s * kTcStageBytes;
+        tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2 + kTcOctets * K * (kTcBitsRow * kOctet + 16));
+        tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
+        tc_tma_load_2d(st + kTcXBytes + kTcWBytes, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
+        tc_tma_load_2d(st + kTcXBytes + kTcWBytes + kTcBitsBytes, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
+                       r0 / kOctet, &full_x[s]);
       }
     }
   } else if (warp == 1) {
@@ -301,7 +291,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
         const uint32_t ws = xs + kTcXBytes;
 #pragma unroll
         for (int kk = 0; kk < kTcBK / 16; ++kk)
-          tc_mma(tmem, tc_desc_sw128(ws + kk * 32), tc_desc_sw128(xs + kk * 32), (kb > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem, tc_desc_sw128(ws + kk * 32), tc_desc_sw128(xs + kk * 32), p.idesc, (kb > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[s]);
       }
       if (ok) tc_commit(done);
@@ -309,16 +299,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
   } else {
     // ---- unpack warps ----
     const int tid = threadIdx.x - 64;
-    UnpackRegs<K> cur, nxt;
-    tc_load_unpack<K>(p, r0, 0, tid, cur);
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % kTcStages;
-      if (kb + 1 < nkb) tc_load_unpack<K>(p, r0, kb + 1, tid, nxt);
-      if (kb >= kTcStages && !tc_wait(&empty[s], unsigned((kb / kTcStages) - 1) & 1u)) { ok = false; break; }
-      tc_store_unpack<K>(smem + s * kTcStageBytes + kTcXBytes, tid, cur);
+      // the stage's TMA loads landing also means its previous MMAs are done
+      if (!tc_wait(&full_x[s], unsigned(kb / kTcStages) & 1u)) { ok = false; break; }
+      unsigned char* st = smem + s * kTcStageBytes;
+      tc_unpack_from_smem<K>(st + kTcXBytes + kTcWBytes, st + kTcXBytes + kTcWBytes + kTcBitsBytes,
+                             st + kTcXBytes, tid);
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
       tc_arrive(&full_w[s]);
-      cur = nxt;
     }
   }
 
@@ -335,22 +324,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, TcParams p) {
       const int quarter = warp & 3;
       const int r = r0 + 32 * quarter + lane;
 #pragma unroll 1
-      for (int c = 0; c < kTcTokens; c += 32) {
-        uint32_t v[32];
+      for (int c = 0; c < p.n_tile; c += 16) {
+        uint32_t v[16];
         const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(c);
         asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-              "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-              "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-              "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+              "=r"(v[15])
             : "r"(taddr));
         asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
         if (r < p.s.M) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int t = t0 + c + j;
             if (t < p.T)
               p.Y[size_t(t) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
@@ -410,7 +396,8 @@ unsigned gemm_error_flags() {
 }
 
 template <int K>
-static cudaError_t launch_tc_k(const CUtensorMap& map, const TcParams& p, cudaStream_t stream) {
+static cudaError_t launch_tc_k(const CUtensorMap& xm, const CUtensorMap& bm, const CUtensorMap& am,
+                               const TcParams& p, cudaStream_t stream) {
   auto fn = gemm_tc_kernel<K>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -418,9 +405,28 @@ static cudaError_t launch_tc_k(const CUtensorMap& map, const TcParams& p, cudaSt
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((p.s.M + kTcRows - 1) / kTcRows, (p.T + kTcTokens - 1) / kTcTokens);
-  fn<<<grid, kTcThreads, kTcSmem, stream>>>(map, p);
+  dim3 grid((p.s.M + kTcRows - 1) / kTcRows, (p.T + p.n_tile - 1) / p.n_tile);
+  fn<<<grid, kTcThreads, kTcSmem, stream>>>(xm, bm, am, p);
   return cudaGetLastError();
+}
+
+// Token tile (MMA N, a multiple of 16 up to 256) that minimises the time of
+// the wave-quantised grid, waves x tile width, for a 128-row tile and one CTA
+// per SM; ties go to the wider tile.
+int tc_token_tile(int M, int T, int sms) {
+  const long long row_tiles = (M + kTcRows - 1) / kTcRows;
+  int best = kTcTokens;
+  long long best_cost = -1;
+  for (int n = kTcTokens; n >= 128; n -= 16) {
+    const long long tiles = row_tiles * ((T + n - 1) / n);
+    const long long waves = (tiles + sms - 1) / sms;
+    const long long cost = waves * n;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = n;
+    }
+  }
+  return best;
 }
 
 // Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
@@ -428,26 +434,49 @@ cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const S
                            int T, uint16_t* Y, cudaStream_t stream) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {cuuint64_t(s.N), cuuint64_t(T)};
-  const cuuint64_t strides[1] = {cuuint64_t(s.N) * 2};
-  const cuuint32_t box[2] = {cuuint32_t(kTcBK), cuuint32_t(kTcTokens)};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  const int n_tile = tc_token_tile(s.M, T, device_sm_count());
+  const cuuint32_t ones[2] = {1, 1};
+  CUtensorMap xm, bm, am;
+  {  // X: bf16 [T][N], box 64 columns x 256 tokens, 128-byte swizzle
+    const cuuint64_t dims[2] = {cuuint64_t(s.N), cuuint64_t(T)};
+    const cuuint64_t strides[1] = {cuuint64_t(s.N) * 2};
+    const cuuint32_t box[2] = {cuuint32_t(kTcBK), cuuint32_t(n_tile)};
+    if (enc(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {  // bits: bytes [O*K][N] (one row = one (octet, kernel)), box 64 bytes x 16K rows
+    const cuuint64_t dims[2] = {cuuint64_t(s.N), cuuint64_t(s.O) * s.K};
+    const cuuint64_t strides[1] = {cuuint64_t(s.N)};
+    const cuuint32_t box[2] = {cuuint32_t(kTcBitsRow * kOctet), cuuint32_t(kTcOctets * s.K)};
+    if (enc(&bm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {  // scales: fp16 [O][G*K*8], box K*8 values x 16 octets
+    const cuuint64_t dims[2] = {cuuint64_t(s.G) * s.K * kOctet, cuuint64_t(s.O)};
+    const cuuint64_t strides[1] = {cuuint64_t(s.G) * s.K * kOctet * 2};
+    const cuuint32_t box[2] = {cuuint32_t(s.K * kOctet), cuuint32_t(kTcOctets)};
+    if (enc(&am, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(alpha), dims, strides, box, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   TcParams p;
   p.packed = packed;
   p.alpha = alpha;
   p.Y = Y;
   p.s = s;
   p.T = T;
+  p.n_tile = n_tile;
+  p.idesc = tc_idesc(n_tile);
   switch (s.K) {
-    case 1: return launch_tc_k<1>(map, p, stream);
-    case 2: return launch_tc_k<2>(map, p, stream);
-    case 3: return launch_tc_k<3>(map, p, stream);
-    default: return launch_tc_k<4>(map, p, stream);
+    case 1: return launch_tc_k<1>(xm, bm, am, p, stream);
+    case 2: return launch_tc_k<2>(xm, bm, am, p, stream);
+    case 3: return launch_tc_k<3>(xm, bm, am, p, stream);
+    default: return launch_tc_k<4>(xm, bm, am, p, stream);
   }
 }
 
