@@ -7,23 +7,28 @@
 // tensor cores read it.  Once decoded the product is a dense contraction, so
 // it runs as bf16 x bf16 -> fp32 MMAs.
 //
-// CTA tile: 128 weight rows (MMA M) x 256 tokens (MMA N), K-steps of 64
-// columns, a 4-stage shared-memory ring.  Per stage:
+// Persistent CTAs (one per SM) walk the tiles of 256 weight rows x n tokens
+// (n <= 256, chosen on the host against wave quantisation) in K-steps of 64
+// columns through a 3-stage shared-memory ring.  The 256 rows are two M=128
+// MMAs that share each X tile, which halves the X traffic through L2 per
+// flop (measured: with 128-row tiles the X re-reads, not the tensor cores or
+// the unpack, bounded the kernel).  Per stage:
 //   * X tile, 256 tokens x 64 columns bf16 (32 KB): one TMA tensor load with
 //     128-byte swizzle; the tile's packed bits (16 octets x K x 64 bytes) and
 //     scales (16 octets x K x 8 fp16) come with two more TMA loads (warp 0);
-//   * W tile, 128 rows x 64 columns bf16 (16 KB): written by 16 unpack warps
-//     (one row x 16 columns per thread) in the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
+//   * W tile, 256 rows x 64 columns bf16 (32 KB): written by 16 unpack warps
+//     (two rows x 16 columns per thread) in the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
 //     the two sign bits are brought to bit 15 and bit 31 by one shift of
 //     (h | h << 15), where h holds the row's 16 bits of one kernel, and
 //     applied to the bf16 scale pair with one LOP3; the K kernels are summed
 //     with packed bf16 adds (HADD2);
-//   * one thread (warp 1) issues 4 tcgen05.mma (M=128, N=256, K=16) into the
-//     tensor-memory accumulator and commits them to the stage's "empty"
-//     barrier.
-// The epilogue (4 warps, one per 32-lane quarter of tensor memory) reads the
-// accumulator with tcgen05.ld: TMEM lane = weight row, column = token, so a
-// warp's 32 lanes store 32 consecutive elements of one output row of Y.
+//   * one thread (warp 1) issues 2 x 4 tcgen05.mma (M=128, N=n, K=16), one
+//     set per row half, into the tensor-memory accumulators and commits them
+//     to the stage's "empty" barrier.
+// The two row halves accumulate in tensor-memory columns 0.. and 256..; 4
+// dedicated epilogue warps (one per 32-lane quarter) drain them.  TMEM lane =
+// weight row, column = token, so a warp's 32 lanes store 32 consecutive
+// elements of one output row of Y.
 // Every mbarrier wait is bounded (1 s); on timeout the CTA records an error
 // flag, drains what it issued (bounded), frees its tensor memory and exits.
 #include <cuda.h>
@@ -32,27 +37,29 @@
 
 namespace mbok {
 
-constexpr int kTcRows = 128;      // weight rows per CTA (MMA M)
+constexpr int kTcRows = 256;      // weight rows per CTA: two M=128 MMAs share each X tile
+constexpr int kTcHalf = 128;      // MMA M
 constexpr int kTcTokens = 256;    // largest token tile per CTA (MMA N); the host picks <= this
 constexpr int kTcBK = 64;         // columns per stage (one 128-byte swizzle row)
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 3;
 constexpr int kTcXBytes = kTcTokens * kTcBK * 2;   // 32 KB
-constexpr int kTcWBytes = kTcRows * kTcBK * 2;     // 16 KB
-constexpr int kTcOctets = kTcRows / kOctet;        // 16 row octets per tile
+constexpr int kTcWBytes = kTcRows * kTcBK * 2;     // 32 KB (two 16 KB halves)
+constexpr int kTcOctets = kTcRows / kOctet;        // 32 row octets per tile
 constexpr int kTcBitsRow = kTcBK / 8;              // 64 columns = 8 bytes per row = 64 bytes per octet
-constexpr int kTcBitsBytes = kTcOctets * MBOK_MAX_K * kTcBitsRow * kOctet;   // 4 KB (K = 4)
-constexpr int kTcAlphaBytes = kTcOctets * MBOK_MAX_K * 16;                 // 1 KB (K = 4)
+constexpr int kTcBitsBytes = kTcOctets * MBOK_MAX_K * kTcBitsRow * kOctet;   // 8 KB (K = 4)
+constexpr int kTcAlphaBytes = kTcOctets * MBOK_MAX_K * 16;                 // 2 KB (K = 4)
 constexpr int kTcStageBytes = kTcXBytes + kTcWBytes + kTcBitsBytes + kTcAlphaBytes;
 constexpr int kTcUnpackWarps = 16;
-constexpr int kTcThreads = (2 + kTcUnpackWarps) * 32;          // TMA, MMA, 16 unpack
+constexpr int kTcEpiWarp0 = 2 + kTcUnpackWarps;                 // 4 epilogue warps follow the unpack warps
+constexpr int kTcThreads = (2 + kTcUnpackWarps + 4) * 32;       // TMA, MMA, 16 unpack, 4 epilogue
 constexpr int kTcSmem = kTcStages * kTcStageBytes + 1024 + 256;  // + alignment + barriers
-constexpr unsigned kTcTmemCols = 256;
+constexpr unsigned kTcTmemCols = 512;      // row halves 0 and 1: columns 0.. and 256..
 constexpr unsigned long long kTcWaitNs = 1000000000ull;
 constexpr unsigned long long kTcDrainNs = 200000000ull;
 
 // Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=n.
 inline uint32_t tc_idesc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTcRows >> 4) << 24);
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTcHalf >> 4) << 24);
 }
 
 __device__ unsigned int g_gemm_error;
@@ -231,17 +238,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                const __grid_constant__ CUtensorMap amap, TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // TMA data landed
-  uint64_t* full_w = full_x + kTcStages;
-  uint64_t* empty = full_w + kTcStages;
-  uint64_t* done = empty + kTcStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // stage's TMA data landed
+  uint64_t* full_w = full_x + kTcStages;   // stage's W tile unpacked
+  uint64_t* empty = full_w + kTcStages;    // stage's MMAs done
+  uint64_t* tfull = empty + kTcStages;     // accumulator b holds a finished tile
+  uint64_t* tempty = tfull + 2;            // accumulator b drained by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = blockIdx.x * kTcRows;
-  const int t0 = blockIdx.y * p.n_tile;
   const int nkb = p.s.N / kTcBK;
+  const int row_tiles = (p.s.M + kTcRows - 1) / kTcRows;
+  const int ntiles = row_tiles * ((p.T + p.n_tile - 1) / p.n_tile);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
@@ -249,7 +257,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       tc_mbar_init(&full_w[s], kTcUnpackWarps * 32);
       tc_mbar_init(&empty[s], 1);
     }
-    tc_mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc_mbar_init(&tfull[b], 1);
+      tc_mbar_init(&tempty[b], 4 * 32);
+    }
     s_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -265,91 +276,113 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
+  // Tile i of this CTA is tile blockIdx.x + i * gridDim.x; row tiles vary
+  // fastest, so CTAs that run together share their X tile through L2.
   if (warp == 0) {
-    // ---- TMA producer: X tiles ----
+    // ---- TMA producer ----
     if (lane == 0) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % kTcStages;
-        if (kb >= kTcStages && !tc_wait(&empty[s], unsigned((kb / kTcStages) - 1) & 1u)) { ok = false; break; }
-        unsigned char* st = smem + s * kTcStageBytes;
-        tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2 + kTcOctets * K * (kTcBitsRow * kOctet + 16));
-        tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
-        tc_tma_load_2d(st + kTcXBytes + kTcWBytes, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
-        tc_tma_load_2d(st + kTcXBytes + kTcWBytes + kTcBitsBytes, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
-                       r0 / kOctet, &full_x[s]);
+      int g = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int r0 = (tile % row_tiles) * kTcRows, t0 = (tile / row_tiles) * p.n_tile;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kTcStages;
+          if (g >= kTcStages && !tc_wait(&empty[s], unsigned((g / kTcStages) - 1) & 1u)) { ok = false; break; }
+          unsigned char* st = smem + s * kTcStageBytes;
+          tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2 + kTcOctets * K * (kTcBitsRow * kOctet + 16));
+          tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
+          tc_tma_load_2d(st + kTcXBytes + kTcWBytes, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
+          tc_tma_load_2d(st + kTcXBytes + kTcWBytes + kTcBitsBytes, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
+                         r0 / kOctet, &full_x[s]);
+        }
       }
     }
   } else if (warp == 1) {
     // ---- MMA issuer ----
     if (lane == 0) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % kTcStages;
-        const unsigned ph = unsigned(kb / kTcStages) & 1u;
-        if (!tc_wait(&full_x[s], ph) || !tc_wait(&full_w[s], ph)) { ok = false; break; }
+      int g = 0, i = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
+        if (i > 0 && !tc_wait(&tempty[0], unsigned(i - 1) & 1u)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t xs = tc_smem(smem + s * kTcStageBytes);
-        const uint32_t ws = xs + kTcXBytes;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kTcStages;
+          const unsigned ph = unsigned(g / kTcStages) & 1u;
+          if (!tc_wait(&full_x[s], ph) || !tc_wait(&full_w[s], ph)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t xs = tc_smem(smem + s * kTcStageBytes);
+          const uint32_t ws = xs + kTcXBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 16; ++kk)
-          tc_mma(tmem, tc_desc_sw128(ws + kk * 32), tc_desc_sw128(xs + kk * 32), p.idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[s]);
+          for (int kk = 0; kk < kTcBK / 16; ++kk) {
+            const uint64_t bdesc = tc_desc_sw128(xs + kk * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + h * (kTcHalf * 128) + kk * 32), bdesc, p.idesc,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[0]);
       }
-      if (ok) tc_commit(done);
     }
-  } else {
+  } else if (warp < kTcEpiWarp0) {
     // ---- unpack warps ----
     const int tid = threadIdx.x - 64;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kTcStages;
-      // the stage's TMA loads landing also means its previous MMAs are done
-      if (!tc_wait(&full_x[s], unsigned(kb / kTcStages) & 1u)) { ok = false; break; }
-      unsigned char* st = smem + s * kTcStageBytes;
-      tc_unpack_from_smem<K>(st + kTcXBytes + kTcWBytes, st + kTcXBytes + kTcWBytes + kTcBitsBytes,
-                             st + kTcXBytes, tid);
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
-      tc_arrive(&full_w[s]);
+    int g = 0;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb, ++g) {
+        const int s = g % kTcStages;
+        // the stage's TMA loads landing also means its previous MMAs are done
+        if (!tc_wait(&full_x[s], unsigned(g / kTcStages) & 1u)) { ok = false; break; }
+        unsigned char* st = smem + s * kTcStageBytes;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          tc_unpack_from_smem<K>(st + kTcXBytes + kTcWBytes, st + kTcXBytes + kTcWBytes + kTcBitsBytes,
+                                 st + kTcXBytes, tid + j * kTcUnpackWarps * 32);
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
+        tc_arrive(&full_w[s]);
+      }
+    }
+  } else {
+    // ---- epilogue warps: TMEM quarter (warp & 3) of both row halves ----
+    const int quarter = warp & 3;
+    int i = 0;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
+      if (!tc_wait(&tfull[0], unsigned(i) & 1u)) { ok = false; break; }
+      tc_fence_after();
+      const int t0 = (tile / row_tiles) * p.n_tile;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int r = (tile % row_tiles) * kTcRows + h * kTcHalf + 32 * quarter + lane;
+#pragma unroll 1
+        for (int c = 0; c < p.n_tile; c += 16) {
+          uint32_t v[16];
+          const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(h * 256 + c);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                "=r"(v[15])
+              : "r"(taddr));
+          asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+          if (r < p.s.M) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int t = t0 + c + j;
+              if (t < p.T)
+                p.Y[size_t(t) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      tc_arrive(&tempty[0]);
     }
   }
 
   if (!ok) atomicOr(&s_fail, 1);
-  __syncthreads();
-  bool fail = s_fail != 0;
-
-  // ---- epilogue: warps 4..7 read TMEM quarter (warp & 3) ----
-  if (!fail && warp >= 4 && warp < 8) {
-    if (!tc_wait(done, 0)) {
-      atomicOr(&s_fail, 1);
-    } else {
-      tc_fence_after();
-      const int quarter = warp & 3;
-      const int r = r0 + 32 * quarter + lane;
-#pragma unroll 1
-      for (int c = 0; c < p.n_tile; c += 16) {
-        uint32_t v[16];
-        const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(c);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-              "=r"(v[15])
-            : "r"(taddr));
-        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-        if (r < p.s.M) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = t0 + c + j;
-            if (t < p.T)
-              p.Y[size_t(t) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
-          }
-        }
-      }
-    }
-  }
-
   tc_fence_before();
   __syncthreads();
-  fail = s_fail != 0;
-  if (fail && threadIdx.x == 0) {
+  if (s_fail != 0 && threadIdx.x == 0) {
     // Record the failure and let every copy and MMA this CTA issued complete
     // (bounded) before its shared memory and tensor memory are released.
     atomicOr(&g_gemm_error, 1u);
@@ -358,6 +391,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       (void)tc_wait(&full_x[s], 1u, kTcDrainNs);
       (void)tc_wait(&empty[s], 0u, kTcDrainNs);
       (void)tc_wait(&empty[s], 1u, kTcDrainNs);
+    }
+    for (int b = 0; b < 2; ++b) {
+      (void)tc_wait(&tfull[b], 0u, kTcDrainNs);
+      (void)tc_wait(&tfull[b], 1u, kTcDrainNs);
     }
   }
   __syncthreads();
@@ -405,7 +442,8 @@ static cudaError_t launch_tc_k(const CUtensorMap& xm, const CUtensorMap& bm, con
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((p.s.M + kTcRows - 1) / kTcRows, (p.T + p.n_tile - 1) / p.n_tile);
+  const int tiles = ((p.s.M + kTcRows - 1) / kTcRows) * ((p.T + p.n_tile - 1) / p.n_tile);
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   fn<<<grid, kTcThreads, kTcSmem, stream>>>(xm, bm, am, p);
   return cudaGetLastError();
 }
