@@ -175,6 +175,21 @@ def cpu_oracle_rate(seconds: float = 10.0):
                       f"4096x4096 layer ({n_rows} rows, {dt:.1f} s); numpy fp64"}
 
 
+def replica_max_ms(ms: float, dist=None, device=None) -> float:
+    """Max over ranks of a per-rank device time (replicas run the same step)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -294,11 +309,9 @@ def run_gpu(a):
         ms, graph = time_graph(torch, step, a.steps, a.warmup, stream)
     clocks = clk.summary()
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = replica_max_ms(ms, dist, dev)
         dist.barrier()
-    value = world * L * bytes_per_layer / (ms * 1e-3) / 1e9
+    value = replica_rate(L * bytes_per_layer, ms, world) / 1e9
     us_per_layer = 1e3 * ms / L
     achieved = bytes_per_layer / (us_per_layer * 1e-6) / 1e9
     traffic = ncu_traffic("gemv_lut.cu", "gemv_lut8_q_proj_k3_4096x4096")
@@ -329,10 +342,8 @@ def run_gpu(a):
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1) / a.steps
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * L * bytes_per_layer / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+        e2e_ms = replica_max_ms(e2e_ms, dist, dev)
+    e2e = {"value": replica_rate(L * bytes_per_layer, e2e_ms, world) / 1e9, "unit": UNIT,
            "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
            "ms_per_step": e2e_ms, "path": "mbok_gemv via the C ABI, pinned host x/y, copies in the timed region"}
 
