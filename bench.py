@@ -423,9 +423,14 @@ def run_gemm_row(torch, mb, wl, dev, peaks, stream, g, out):
 
 
 def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
-    # Small batch, LLaMA-7B gate 11008 x 4096, K=3 (and down 4096 x 11008, K=2).
-    for (name, K, M, N) in (("gate", 3, 11008, 4096), ("down", 2, 4096, 11008)):
-        L = 8
+    # Batch 1 / 4 / 16 on LLaMA-7B shapes (q_proj 4096x4096 K=3, gate 11008x4096
+    # K=3, down 4096x11008 K=2), each on both GEMV kernels.  Enough distinct
+    # weight copies per graph that they exceed L2 (>= 150 MB).
+    shapes = (("q_proj", 3, 4096, 4096), ("gate", 3, 11008, 4096), ("down", 2, 4096, 11008))
+    kernels = (("lookup", mb.GEMV_LOOKUP), ("tensor", mb.GEMV_TENSOR))
+    for (name, K, M, N) in shapes:
+        bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
+        L = max(8, -(-150_000_000 // bpl))
         packed = [torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
                                 device=dev, generator=g) for _ in range(L)]
         al = []
@@ -435,19 +440,23 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
                           .view(torch.float16), K, M, N, t)
             al.append(t)
         ws = mb.zeros_workspace(K, M, N, 16, dev)
-        bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
         for batch in (1, 4, 16):
             x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
             y = torch.empty(batch, M, dtype=torch.float32, device=dev)
+            for (kname, kcode) in kernels:
+                if name == "q_proj" and batch > 1 and kname == "lookup":
+                    continue
 
-            def fn():
-                for l in range(L):
-                    mb.gemv(packed[l], al[l], K, M, N, 128, x, mb.BF16, batch, y, ws, stream=stream)
-            ms, gr = time_graph(torch, fn, 10, 3, stream)
-            gbs = L * bpl / (ms * 1e-3) / 1e9
-            out[f"gemv_llama7b_{name}_k{K}_{M}x{N}_b{batch}"] = {
-                "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
-            del gr
+                def fn():
+                    for l in range(L):
+                        mb.gemv(packed[l], al[l], K, M, N, 128, x, mb.BF16, batch, y, ws, stream=stream)
+                with mb.gemv_kernel(kcode):
+                    ms, gr = time_graph(torch, fn, 10, 3, stream)
+                gbs = L * bpl / (ms * 1e-3) / 1e9
+                out[f"gemv_llama7b_{name}_k{K}_{M}x{N}_b{batch}_{kname}"] = {
+                    "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                    "layers": L}
+                del gr
         del packed, al
         torch.cuda.empty_cache()
 

@@ -22,6 +22,9 @@ BF16 = 1
 GROUP = 128
 MAX_K = 4
 MAX_BATCH = 16
+GEMV_AUTO = 0
+GEMV_LOOKUP = 1
+GEMV_TENSOR = 2
 
 _lib = None
 
@@ -54,6 +57,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
+            "mbok_gemv_set_kernel": ([i], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -159,6 +163,28 @@ def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=Non
     library's built-in array (see include/mbok.h)."""
     _check(lib().mbok_gemv_noalloc(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype,
                                    batch, _ptr(y), _stream(stream)), "mbok_gemv_noalloc")
+
+
+def gemv_set_kernel(kernel: int) -> None:
+    """Process-wide kernel choice of gemv / gemv_noalloc (GEMV_AUTO,
+    GEMV_LOOKUP or GEMV_TENSOR)."""
+    _check(lib().mbok_gemv_set_kernel(kernel), "mbok_gemv_set_kernel")
+
+
+class gemv_kernel:
+    """Context manager: run the enclosed gemv calls on one kernel, then
+    return to GEMV_AUTO."""
+
+    def __init__(self, kernel: int):
+        self.kernel = kernel
+
+    def __enter__(self):
+        gemv_set_kernel(self.kernel)
+        return self
+
+    def __exit__(self, *exc):
+        gemv_set_kernel(GEMV_AUTO)
+        return False
 
 
 def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:

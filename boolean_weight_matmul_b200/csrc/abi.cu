@@ -12,9 +12,34 @@ cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const
                             float*, void*, cudaStream_t);
 size_t gemv_lut_workspace_bytes(const Shape&);
 unsigned gemv_error_flags();
+unsigned gemv_mma_error_flags();
+cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int,
+                            float*, cudaStream_t);
+cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
+                        void*, cudaStream_t);
 cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
                            uint16_t*, cudaStream_t);
 unsigned gemm_error_flags();
+
+// Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc.
+int gemv_kernel_choice = MBOK_GEMV_AUTO;
+
+// One decode GEMV call: the lookup-table kernel once per vector, or the
+// tensor-core kernel over the whole batch.
+cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
+                        bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
+  bool tensor = batch > 1;
+  if (gemv_kernel_choice == MBOK_GEMV_LOOKUP) tensor = false;
+  if (gemv_kernel_choice == MBOK_GEMV_TENSOR) tensor = true;
+  if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream);
+  const size_t xbytes = x_f32 ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    const void* xb = static_cast<const char*>(x) + size_t(b) * s.N * xbytes;
+    const cudaError_t e = launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 }  // namespace mbok
 
 using namespace mbok;
@@ -123,14 +148,13 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
   const size_t need = gemv_lut_workspace_bytes(s);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
     return MBOK_ERR_WORKSPACE;
-  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
-  for (int b = 0; b < batch; ++b) {
-    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
-    const cudaError_t e = launch_gemv_lut(reinterpret_cast<const uint8_t*>(packed), alpha, s, xb,
-                                          x_dtype == MBOK_F32, y + size_t(b) * M, workspace,
-                                          as_stream(stream));
-    if (e != cudaSuccess) return MBOK_ERR_CUDA;
-  }
+  return from_cuda(launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32,
+                               batch, y, workspace, as_stream(stream)));
+}
+
+int mbok_gemv_set_kernel(int kernel) {
+  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TENSOR) return MBOK_ERR_INVALID_ARG;
+  gemv_kernel_choice = kernel;
   return MBOK_OK;
 }
 
@@ -139,8 +163,9 @@ int mbok_read_device_errors(unsigned* flags) {
   if (cudaDeviceSynchronize() != cudaSuccess) return MBOK_ERR_CUDA;
   const unsigned g = gemv_error_flags();
   const unsigned m = gemm_error_flags();
-  if (g == ~0u || m == ~0u) return MBOK_ERR_CUDA;
-  *flags = (g ? 1u : 0u) | (m ? 2u : 0u);
+  const unsigned t = gemv_mma_error_flags();
+  if (g == ~0u || m == ~0u || t == ~0u) return MBOK_ERR_CUDA;
+  *flags = (g ? 1u : 0u) | (m ? 2u : 0u) | (t ? 4u : 0u);
   return MBOK_OK;
 }
 

@@ -1,0 +1,508 @@
+// Small-batch GEMV Y = W X for 1..16 activation vectors on tensor cores, sm_100a.
+//
+// The layer is y_r = sum_g sum_k alpha_{k,r,g} * s_{k,r,g} with
+// s_{k,r,g} = sum_{j in g} b_{k,r,j} x_j, b in {-1,+1} (Paper-Notes page,
+// 方法详解 / 关键设计: W x as K Boolean products, one scale per group).  For
+// more than one vector the per-bit work of a lookup table grows with the
+// batch, so this kernel computes the K Boolean products s_{k,.,g} as exact
+// tensor-core products instead:
+//
+//  * A = the +-1 signs of one kernel for 16 rows x 16 columns, built in
+//    registers as bf16 pairs (0x3F80 = +1, 0xBF80 = -1): each pair is one
+//    shift and one three-input logic op on the bit pattern.  Signs are exact
+//    in bf16, bf16 activations are exact, and products are exact in the fp32
+//    accumulator, so every s_{k,r,g} is an fp32 sum of exact terms.
+//  * B = the activations: column n of the 8-wide MMA tile is vector n.  fp32
+//    activations are split exactly into three bf16 parts (hi + mid + lo) that
+//    take three columns; their results are added back at the end.
+//  * One m16n8k16 MMA per (kernel, 16 columns, 8 columns of B); after each
+//    128-column group the fp32 result is scaled by the group's fp16 scales
+//    and added into the output accumulators (fp32 FMA), so the scales are
+//    applied exactly as the method's grouped sum states.
+//  * A CTA owns one 16-row tile (two storage octets) and all N columns.  The
+//    tile's bits and scales and the activations stream through a 4-stage
+//    shared-memory ring in column slices (1024 columns; 512 when B has 16
+//    columns): per slice, one bulk asynchronous copy per (octet, kernel) (the
+//    slice is contiguous in storage format 1), one per octet for the scales
+//    and one per activation vector, all completing on the stage's mbarrier.
+//    The 8 warps split a slice's 64-column chunks; their partial sums meet in
+//    shared memory, summed in warp order: no cross-CTA combine, no
+//    workspace, deterministic.
+//  * The k-index of an MMA is a permutation of the 16 columns it covers:
+//    thread (g, t) of a warp reads the halfword of row g for unit 4c + t of
+//    chunk c, and MMA j of the chunk takes bits 4j..4j+3 of it (columns
+//    16(4c+t) + 4j .. +3).  B uses the same permutation, which is simply 16
+//    consecutive activations of that unit per thread (vector rows padded by
+//    16 bytes in shared memory so these reads are conflict-free).
+//  * Launches use programmatic dependent launch: before waiting on the
+//    previous grid a CTA only asks L2 to prefetch its tile's bits and scales.
+//  * Every mbarrier wait is bounded (1 s); on timeout the CTA records an
+//    error flag (bit 2 of mbok_read_device_errors), skips the rest of its
+//    work, waits (bounded) for its copies in flight and exits without
+//    storing.
+#include "mbok_common.cuh"
+
+namespace mbok {
+
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kChunkCols = 64;                      // 4 units, 4 MMAs per kernel
+constexpr int kMmaStages = 4;
+constexpr int kMaxNT = 2;                           // up to 16 columns of B per launch
+constexpr unsigned long long kMmaWaitNs = 1000000000ull;
+constexpr unsigned long long kMmaDrainNs = 200000000ull;
+
+// One ring stage: a slice of kCols columns of the tile's two octets (bits of
+// every kernel, scales) and of every activation vector.  Narrower slices when
+// B has 16 columns keep the activations' share of a stage bounded.
+template <int K, int NT, bool XF32>
+struct MmaGeom {
+  static constexpr int kCols = NT == 1 ? 1024 : 512;
+  static constexpr int kUnits = kCols / kUnit;
+  static constexpr int kGroups = kCols / kGroup;
+  static constexpr int kXElem = XF32 ? 4 : 2;
+  static constexpr int kMaxVec = XF32 ? (8 * NT) / 3 : 8 * NT;
+  static constexpr int kXStride = kCols * kXElem + 16;          // padded: conflict-free B reads
+  static constexpr int kBits = 2 * K * kUnits * 16;             // [octet][k][unit][8 rows][2 B]
+  static constexpr int kAlpha = 2 * kGroups * K * 16;           // [octet][group][k][8 rows][2 B]
+  static constexpr int kRed = kMmaWarps * NT * 8 * 16 * 4;
+  // [bits | scales | nb activation rows]; the ring holds kMmaStages of these.
+  static constexpr int stage_bytes(int nb) { return kBits + kAlpha + nb * kXStride; }
+  static constexpr int smem_bytes(int nb) { return kMmaStages * stage_bytes(nb) + kRed; }
+};
+
+__device__ unsigned int g_gemv_mma_error;
+
+struct GemvMmaParams {
+  const uint8_t* packed;
+  const uint16_t* alpha;
+  const void* x;        // [nb][N] bf16 or fp32
+  float* y;             // [nb][M]
+  Shape s;
+  int nb;               // vectors in this launch
+  uint32_t mul[8];      // 2^(15 - 2i): sign_pair factors
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t mm_smem(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long mm_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void grid_dependency_wait_mma() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents_mma() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mm_bar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(mm_smem(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mm_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(mm_smem(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mm_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(mm_smem(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false on timeout.
+__device__ __forceinline__ bool mm_wait(uint64_t* bar, unsigned parity, unsigned long long limit) {
+  const uint32_t a = mm_smem(bar);
+  unsigned long long t0 = 0;
+  for (unsigned it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 255u) == 0) {
+      const unsigned long long t = mm_ns();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > limit) return false;
+    }
+  }
+}
+
+// Bulk copy global -> this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          mm_smem(dst)),
+      "l"(src), "r"(bytes), "r"(mm_smem(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------------
+// Operands
+// ---------------------------------------------------------------------------
+
+// Bits p and p+1 of the halfword h as a bf16 pair of signs (+1 for a set
+// bit).  u = h | h << 15 holds bit p at p and bit p+1 at p+16.  The pair is
+// (~u & (0x80008000 >> s)) * 2^s + 0x3F803F80 with s = 15 - p: the two
+// isolated (inverted) bits land on the sign positions of 1.0 / 1.0 without
+// carries.  One logic op (ALU pipe) and one integer multiply-add; the factor
+// 2^s comes from the kernel parameters (mul[p/2]) so that the multiply-add
+// stays an IMAD on the FMA pipe instead of becoming a shift on the ALU pipe.
+template <int P>
+__device__ __forceinline__ uint32_t sign_pair(uint32_t u, const uint32_t* mul) {
+  static_assert(P % 2 == 0 && P < 15, "pairs start at an even bit below 15");
+  constexpr uint32_t kMask = 0x80008000u >> (15 - P);
+  return (~u & kMask) * mul[P / 2] + 0x3F803F80u;
+}
+
+__device__ __forceinline__ uint32_t spread(uint32_t h) { return h | (h << 15); }
+
+__device__ __forceinline__ uint32_t f32_to_bf16_rn(float v) {
+  return uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+}
+
+// Part `part` (0 = hi, 1 = mid, 2 = lo) of the exact three-way bf16 split of v.
+__device__ __forceinline__ uint32_t bf16_part(float v, int part) {
+  const uint32_t h = f32_to_bf16_rn(v);
+  if (part == 0) return h;
+  const float r = __fsub_rn(v, __uint_as_float(h << 16));
+  const uint32_t m = f32_to_bf16_rn(r);
+  if (part == 1) return m;
+  return f32_to_bf16_rn(__fsub_rn(r, __uint_as_float(m << 16)));
+}
+
+// The B fragment words of one chunk for column n of B: the 16 activations of
+// unit uq of the stage's slice, vector n (or n/3, part n%3, for fp32), as 8
+// bf16 pairs; zeros for unused columns.
+template <bool XF32, int XS>
+__device__ __forceinline__ void load_b(const unsigned char* xs, int nb, int n, int uq, uint32_t b[8]) {
+  const int vec = XF32 ? n / 3 : n;
+  if (vec >= nb) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = 0u;
+    return;
+  }
+  if (!XF32) {
+    const uint4* src = reinterpret_cast<const uint4*>(xs + vec * XS + uq * kUnit * 2);
+    const uint4 v0 = src[0], v1 = src[1];
+    b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
+    b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
+  } else {
+    const int part = n - 3 * vec;
+    const float4* src = reinterpret_cast<const float4*>(xs + vec * XS + uq * kUnit * 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = src[i];
+      b[2 * i] = bf16_part(v.x, part) | (bf16_part(v.y, part) << 16);
+      b[2 * i + 1] = bf16_part(v.z, part) | (bf16_part(v.w, part) << 16);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+
+// Thread 0: copy slice `sl` of the tile (octets o0, o0+1) and of the
+// activations into a ring stage.
+template <int K, int NT, bool XF32>
+__device__ __forceinline__ void issue_slice(const GemvMmaParams& p, int o0, int n_oct, int sl, unsigned char* stage,
+                                            uint64_t* full) {
+  using G = MmaGeom<K, NT, XF32>;
+  const Shape& s = p.s;
+  const int u0 = sl * G::kUnits;
+  const int nu = min(G::kUnits, s.Q - u0);
+  const int ng = nu / kUnitsPerGroup;
+  const uint32_t bits_bytes = uint32_t(nu) * 16;
+  const uint32_t alpha_bytes = uint32_t(ng) * K * 16;
+  const uint32_t x_bytes = uint32_t(nu) * kUnit * G::kXElem;
+  mm_arrive_expect_tx(full, uint32_t(n_oct) * (K * bits_bytes + alpha_bytes) + uint32_t(p.nb) * x_bytes);
+  for (int oi = 0; oi < n_oct; ++oi) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      bulk_copy(stage + (oi * K + k) * G::kUnits * 16, p.packed + unit_offset(s, o0 + oi, k, u0), bits_bytes, full);
+    bulk_copy(stage + G::kBits + oi * G::kGroups * K * 16, p.alpha + alpha_offset(s, o0 + oi, u0 / kUnitsPerGroup, 0),
+              alpha_bytes, full);
+  }
+  const unsigned char* x = static_cast<const unsigned char*>(p.x);
+  for (int v = 0; v < p.nb; ++v)
+    bulk_copy(stage + G::kBits + G::kAlpha + v * G::kXStride,
+              x + (size_t(v) * s.N + size_t(u0) * kUnit) * G::kXElem, x_bytes, full);
+}
+
+template <int K, int NT, bool XF32>
+__global__ void __launch_bounds__(kMmaThreads, NT == 1 ? 3 : 2) gemv_mma_kernel(GemvMmaParams p) {
+  using G = MmaGeom<K, NT, XF32>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int stage_bytes = G::stage_bytes(p.nb);
+  float (*red)[NT * 8][16] = reinterpret_cast<float (*)[NT * 8][16]>(smem + kMmaStages * stage_bytes);
+  __shared__ __align__(8) uint64_t full[kMmaStages], empty[kMmaStages];
+  __shared__ int s_abort;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const Shape& s = p.s;
+  const int o0 = 2 * blockIdx.x;
+  const int n_oct = (o0 + 1 < s.O) ? 2 : 1;
+  const int n_slices = (s.N + G::kCols - 1) / G::kCols;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMmaStages; ++i) {
+      mm_bar_init(&full[i], 1);
+      mm_bar_init(&empty[i], kMmaWarps);
+    }
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  // Before the dependency wait: L2 prefetch of this tile's bits and scales.
+  if (warp == 1) {
+    const size_t bits_bytes = size_t(n_oct) * s.K * s.N;
+    const size_t alpha_bytes = size_t(n_oct) * s.G * s.K * kOctet * 2;
+    const uint8_t* bsrc = p.packed + unit_offset(s, o0, 0, 0);
+    const uint8_t* asrc = reinterpret_cast<const uint8_t*>(p.alpha + alpha_offset(s, o0, 0, 0));
+    constexpr size_t kPiece = 16384;
+    for (size_t off = size_t(lane) * kPiece; off < bits_bytes; off += 32 * kPiece)
+      bulk_prefetch_l2(bsrc + off, uint32_t(min(kPiece, bits_bytes - off)));
+    if (lane == 31) {
+      for (size_t off = 0; off < alpha_bytes; off += kPiece)
+        bulk_prefetch_l2(asrc + off, uint32_t(min(kPiece, alpha_bytes - off)));
+    }
+  }
+  allow_dependents_mma();
+  grid_dependency_wait_mma();
+  __syncthreads();   // barrier initialisation visible to all threads
+
+  int issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < kMmaStages && issued < n_slices; ++issued)
+      issue_slice<K, NT, XF32>(p, o0, n_oct, issued, smem + issued * stage_bytes, &full[issued]);
+  }
+
+  float yacc[NT][4];
+  float d[K][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      yacc[nt][i] = 0.f;
+#pragma unroll
+      for (int k = 0; k < K; ++k) d[k][nt][i] = 0.f;
+    }
+
+  for (int sl = 0; sl < n_slices; ++sl) {
+    const int st = sl % kMmaStages;
+    const unsigned phase = unsigned(sl / kMmaStages) & 1u;
+    // Every decision below is made warp-uniform (the MMAs are warp-wide).
+    bool good = true;
+    if (warp == 0) {
+      // Refill: slice sl + stages - 1 goes into the stage slice sl - 1 used,
+      // once every warp has released it.
+      if (lane == 0 && sl >= 1 && issued < n_slices) {
+        const int pst = (sl - 1) % kMmaStages;
+        good = mm_wait(&empty[pst], unsigned((sl - 1) / kMmaStages) & 1u, kMmaWaitNs);
+        if (good) {
+          issue_slice<K, NT, XF32>(p, o0, n_oct, issued, smem + pst * stage_bytes, &full[pst]);
+          ++issued;
+        }
+      }
+      good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    }
+    if (good) good = *reinterpret_cast<volatile int*>(&s_abort) == 0;
+    if (good) good = mm_wait(&full[st], phase, kMmaWaitNs);
+    good = __all_sync(0xffffffffu, good);
+    if (!good) {
+      if (lane == 0) {
+        atomicOr(&g_gemv_mma_error, 1u);
+        *reinterpret_cast<volatile int*>(&s_abort) = 1;
+      }
+      break;
+    }
+
+    const unsigned char* bits = smem + st * stage_bytes;
+    const unsigned char* alph = bits + G::kBits;
+    const unsigned char* xs = alph + G::kAlpha;
+    const int u0 = sl * G::kUnits;
+    const int nchunks = min(G::kUnits, s.Q - u0) / 4;
+    const int c_begin = warp * nchunks / kMmaWarps, c_end = (warp + 1) * nchunks / kMmaWarps;
+    int grp = c_begin * kChunkCols / kGroup;
+    for (int c = c_begin; c < c_end; ++c) {
+      const int uq = 4 * c + t;   // unit within the slice
+      uint32_t b[NT][8];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) load_b<XF32, G::kXStride>(xs, p.nb, g + 8 * nt, uq, b[nt]);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
+        const uint32_t h1 = n_oct > 1 ? *reinterpret_cast<const uint16_t*>(bits + ((K + k) * G::kUnits + uq) * 16 + 2 * g)
+                                      : 0u;
+        const uint32_t v0 = spread(h0), v1 = spread(h1);
+        uint32_t a[4][4];
+        a[0][0] = sign_pair<0>(v0, p.mul);  a[0][1] = sign_pair<0>(v1, p.mul);  a[0][2] = sign_pair<2>(v0, p.mul);  a[0][3] = sign_pair<2>(v1, p.mul);
+        a[1][0] = sign_pair<4>(v0, p.mul);  a[1][1] = sign_pair<4>(v1, p.mul);  a[1][2] = sign_pair<6>(v0, p.mul);  a[1][3] = sign_pair<6>(v1, p.mul);
+        a[2][0] = sign_pair<8>(v0, p.mul);  a[2][1] = sign_pair<8>(v1, p.mul);  a[2][2] = sign_pair<10>(v0, p.mul); a[2][3] = sign_pair<10>(v1, p.mul);
+        a[3][0] = sign_pair<12>(v0, p.mul); a[3][1] = sign_pair<12>(v1, p.mul); a[3][2] = sign_pair<14>(v0, p.mul); a[3][3] = sign_pair<14>(v1, p.mul);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[k][nt], a[j], b[nt][2 * j], b[nt][2 * j + 1]);
+      }
+      // End of a 128-column group (or of this warp's part of the slice).
+      const int next_grp = (c + 1) * kChunkCols / kGroup;
+      if (c + 1 == c_end || next_grp != grp) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const float a0 = __half2float(__ushort_as_half(
+              *reinterpret_cast<const uint16_t*>(alph + (grp * K + k) * 16 + 2 * g)));
+          const float a1 = n_oct > 1 ? __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(
+                                           alph + ((G::kGroups + grp) * K + k) * 16 + 2 * g)))
+                                     : 0.f;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            yacc[nt][0] = __fmaf_rn(a0, d[k][nt][0], yacc[nt][0]);
+            yacc[nt][1] = __fmaf_rn(a0, d[k][nt][1], yacc[nt][1]);
+            yacc[nt][2] = __fmaf_rn(a1, d[k][nt][2], yacc[nt][2]);
+            yacc[nt][3] = __fmaf_rn(a1, d[k][nt][3], yacc[nt][3]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[k][nt][i] = 0.f;
+          }
+        }
+        grp = next_grp;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mm_arrive(&empty[st]);
+  }
+
+  // Partial sums of this warp: rows g, g+8, columns 8nt + 2t, 8nt + 2t + 1.
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    red[warp][8 * nt + 2 * t][g] = yacc[nt][0];
+    red[warp][8 * nt + 2 * t + 1][g] = yacc[nt][1];
+    red[warp][8 * nt + 2 * t][g + 8] = yacc[nt][2];
+    red[warp][8 * nt + 2 * t + 1][g + 8] = yacc[nt][3];
+  }
+  __syncthreads();
+  const bool aborted = *reinterpret_cast<volatile int*>(&s_abort) != 0;
+  if (aborted) {
+    // Wait (bounded) for every copy this CTA issued, then leave without storing.
+    if (threadIdx.x == 0) {
+      for (int sl = 0; sl < issued; ++sl)
+        mm_wait(&full[sl % kMmaStages], unsigned(sl / kMmaStages) & 1u, kMmaDrainNs);
+    }
+    return;
+  }
+  // Thread (vector, row): sum over warps in order (and over the three parts
+  // of an fp32 vector, hi + mid first).
+  const int vec = threadIdx.x >> 4, r = threadIdx.x & 15;
+  const int row = 16 * blockIdx.x + r;
+  if (vec < p.nb && row < s.M) {
+    float total;
+    if (!XF32) {
+      total = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMmaWarps; ++w) total += red[w][vec][r];
+    } else {
+      float part[3];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        part[q] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaWarps; ++w) part[q] += red[w][3 * vec + q][r];
+      }
+      total = (part[0] + part[1]) + part[2];
+    }
+    p.y[size_t(vec) * s.M + row] = total;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+template <int K, int NT, bool XF32>
+static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
+  auto fn = gemv_mma_kernel<K, NT, XF32>;
+  using G = MmaGeom<K, NT, XF32>;
+  static bool attr_set = false;   // set once (for the largest batch), outside any stream capture
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               G::smem_bytes(G::kMaxVec));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.s.O + 1) / 2);
+  cfg.blockDim = dim3(kMmaThreads);
+  cfg.dynamicSmemBytes = G::smem_bytes(p.nb);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int K>
+static cudaError_t launch_mma_nt(const GemvMmaParams& p, bool x_f32, cudaStream_t stream) {
+  const int cols = x_f32 ? 3 * p.nb : p.nb;
+  if (cols <= 8) return x_f32 ? launch_mma_k<K, 1, true>(p, stream) : launch_mma_k<K, 1, false>(p, stream);
+  return x_f32 ? launch_mma_k<K, 2, true>(p, stream) : launch_mma_k<K, 2, false>(p, stream);
+}
+
+// Reads and clears the kernel's error flag; ~0u if the read itself failed.
+unsigned gemv_mma_error_flags() {
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gemv_mma_error, sizeof(v)) != cudaSuccess) return ~0u;
+  const unsigned z = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_gemv_mma_error, &z, sizeof(z)) != cudaSuccess) return ~0u;
+  return v;
+}
+
+// Y[b] = W X[b] for b < batch (x: [batch][N], y: [batch][M]); launches cover
+// up to 16 bf16 or 5 fp32 vectors each.
+cudaError_t launch_gemv_mma(const uint8_t* packed, const uint16_t* alpha, const Shape& s,
+                            const void* x, bool x_f32, int batch, float* y, cudaStream_t stream) {
+  const int per_launch = x_f32 ? (8 * kMaxNT) / 3 : 8 * kMaxNT;
+  const size_t x_elem = x_f32 ? 4 : 2;
+  for (int b0 = 0; b0 < batch; b0 += per_launch) {
+    GemvMmaParams p;
+    p.packed = packed;
+    p.alpha = alpha;
+    p.x = static_cast<const char*>(x) + size_t(b0) * s.N * x_elem;
+    p.y = y + size_t(b0) * s.M;
+    p.s = s;
+    p.nb = batch - b0 < per_launch ? batch - b0 : per_launch;
+    for (int i = 0; i < 8; ++i) p.mul[i] = 1u << (15 - 2 * i);
+    cudaError_t e;
+    switch (s.K) {
+      case 1: e = launch_mma_nt<1>(p, x_f32, stream); break;
+      case 2: e = launch_mma_nt<2>(p, x_f32, stream); break;
+      case 3: e = launch_mma_nt<3>(p, x_f32, stream); break;
+      default: e = launch_mma_nt<4>(p, x_f32, stream); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace mbok

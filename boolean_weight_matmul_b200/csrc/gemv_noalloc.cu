@@ -5,6 +5,8 @@
 #include "mbok_common.cuh"
 
 namespace mbok {
+cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
+                        void*, cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t);
 size_t gemv_lut_workspace_bytes(const Shape&);
@@ -69,12 +71,8 @@ extern "C" int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, 
     // The array keeps whatever the previous call left: clear the counters.
     if (cudaMemsetAsync(scratch, 0, kCounterBytesToClear, st) != cudaSuccess) return MBOK_ERR_CUDA;
   }
-  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
-  for (int b = 0; b < batch; ++b) {
-    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
-    if (launch_gemv_lut(reinterpret_cast<const uint8_t*>(packed), alpha, s, xb,
-                        x_dtype == MBOK_F32, y + size_t(b) * M, scratch, st) != cudaSuccess)
-      return MBOK_ERR_CUDA;
-  }
+  if (launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32, batch, y,
+                  scratch, st) != cudaSuccess)
+    return MBOK_ERR_CUDA;
   return MBOK_OK;
 }

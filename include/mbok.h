@@ -62,6 +62,10 @@ typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
 #define MBOK_LAYOUT_VERSION 1
 #define MBOK_MAX_K 4
 #define MBOK_MAX_BATCH 16
+/* Values of mbok_gemv_set_kernel. */
+#define MBOK_GEMV_AUTO 0
+#define MBOK_GEMV_LOOKUP 1
+#define MBOK_GEMV_TENSOR 2
 /* Size of the scratch array built into the library for mbok_gemv_noalloc. */
 #define MBOK_NOALLOC_SCRATCH_BYTES (4u << 20)
 
@@ -128,10 +132,23 @@ int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint3
  *   workspace, workspace_bytes : see mbok_gemv_workspace_bytes.
  * Accuracy: |y - y_exact| <= 1e-3 * sum_j |W[r][j] x[b][j]| + 1e-6 per
  * element and relative L2 error <= 1e-5 (fp32 accumulation).  For a given
- * (shape, batch) the result is deterministic run to run. */
+ * (shape, batch, kernel choice) the result is deterministic run to run.
+ * Kernels (see mbok_gemv_set_kernel): by default one vector runs on the
+ * lookup-table kernel and two or more on the tensor-core kernel, which
+ * forms each +-1 dot product as an exact bf16 MMA (fp32 activations are
+ * split exactly into three bf16 parts) and scales it per group in fp32. */
 int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
               const void* x, int x_dtype, int batch, float* y, void* workspace,
               size_t workspace_bytes, void* stream);
+
+/* Kernel choice of mbok_gemv and mbok_gemv_noalloc for this process (all
+ * devices, all later calls): MBOK_GEMV_AUTO (default: lookup tables for one
+ * vector, tensor cores for more), MBOK_GEMV_LOOKUP (lookup tables, one
+ * launch per vector) or MBOK_GEMV_TENSOR (tensor cores for any batch).  Both
+ * kernels meet the accuracy stated for mbok_gemv; their results differ in
+ * rounding.  Not synchronised with calls in flight on other host threads.
+ * Returns MBOK_ERR_INVALID_ARG for any other value. */
+int mbok_gemv_set_kernel(int kernel);
 
 /* mbok_gemv without a workspace argument, for callers that cannot allocate
  * device memory: code that must not call cudaMalloc after start-up (an
@@ -164,7 +181,8 @@ int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int 
  * a kernel that gives up records a flag and returns early instead of hanging.
  * Writes the flags accumulated on the current device since the last call to
  * *flags (0 = none; bit 0 = a decode-GEMV copy never completed; bit 1 = a
- * prefill-GEMM pipeline wait gave up) and clears them.  Synchronises the
+ * prefill-GEMM pipeline wait gave up; bit 2 = a tensor-core GEMV copy wait
+ * gave up, in which case that launch stored no outputs) and clears them.  Synchronises the
  * device.  Returns MBOK_ERR_CUDA if the flags cannot be read. */
 int mbok_read_device_errors(unsigned* flags);
 

@@ -97,3 +97,14 @@ def test_binding_refuses_cpu_tensors(L):
     s = torch.ones(1, 8, 128, dtype=torch.int8)
     with pytest.raises(ValueError):
         mb.pack_bits(s, 1, 8, 128, torch.empty(64, dtype=torch.int32))
+
+
+def test_gemv_kernel_choice(L):
+    import boolean_weight_matmul_b200 as mb
+    assert L.mbok_gemv_set_kernel(-1) == 1 and L.mbok_gemv_set_kernel(3) == 1
+    for k in (mb.GEMV_LOOKUP, mb.GEMV_TENSOR, mb.GEMV_AUTO):
+        assert L.mbok_gemv_set_kernel(k) == 0
+    with mb.gemv_kernel(mb.GEMV_TENSOR):
+        pass
+    with pytest.raises(mb.MbokError):
+        mb.gemv_set_kernel(7)
