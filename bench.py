@@ -427,7 +427,8 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
     # K=3, down 4096x11008 K=2), each on both GEMV kernels.  Enough distinct
     # weight copies per graph that they exceed L2 (>= 150 MB).
     shapes = (("q_proj", 3, 4096, 4096), ("gate", 3, 11008, 4096), ("down", 2, 4096, 11008))
-    kernels = (("lookup", mb.GEMV_LOOKUP), ("tensor", mb.GEMV_TENSOR))
+    kernels = (("lookup", mb.GEMV_LOOKUP, False), ("lookup_static", mb.GEMV_LOOKUP, True),
+               ("tensor", mb.GEMV_TENSOR, False))
     for (name, K, M, N) in shapes:
         bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
         L = max(8, -(-150_000_000 // bpl))
@@ -443,15 +444,17 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
         for batch in (1, 4, 16):
             x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
             y = torch.empty(batch, M, dtype=torch.float32, device=dev)
-            for (kname, kcode) in kernels:
-                if name == "q_proj" and batch > 1 and kname == "lookup":
+            for (kname, kcode, static) in kernels:
+                if batch > 1 and (kname.endswith("static") or (name == "q_proj" and kname == "lookup")):
                     continue
 
                 def fn():
                     for l in range(L):
                         mb.gemv(packed[l], al[l], K, M, N, 128, x, mb.BF16, batch, y, ws, stream=stream)
+                mb.gemv_set_static_weights(static)
                 with mb.gemv_kernel(kcode):
                     ms, gr = time_graph(torch, fn, 10, 3, stream)
+                mb.gemv_set_static_weights(False)
                 gbs = L * bpl / (ms * 1e-3) / 1e9
                 out[f"gemv_llama7b_{name}_k{K}_{M}x{N}_b{batch}_{kname}"] = {
                     "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],

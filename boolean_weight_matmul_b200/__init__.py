@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
             "mbok_gemv_set_kernel": ([i], i),
+            "mbok_gemv_set_static_weights": ([i], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -169,6 +170,12 @@ def gemv_set_kernel(kernel: int) -> None:
     """Process-wide kernel choice of gemv / gemv_noalloc (GEMV_AUTO,
     GEMV_LOOKUP or GEMV_TENSOR)."""
     _check(lib().mbok_gemv_set_kernel(kernel), "mbok_gemv_set_kernel")
+
+
+def gemv_set_static_weights(on: bool) -> None:
+    """Promise that GEMV weights are never written by work still running
+    when a GEMV launches (see include/mbok.h)."""
+    _check(lib().mbok_gemv_set_static_weights(1 if on else 0), "mbok_gemv_set_static_weights")
 
 
 class gemv_kernel:

@@ -9,7 +9,7 @@ cudaError_t launch_pack_alpha(const uint16_t*, const Shape&, uint16_t*, cudaStre
 cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __half*, float*,
                                      cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
-                            float*, void*, cudaStream_t);
+                            float*, void*, cudaStream_t, bool);
 size_t gemv_lut_workspace_bytes(const Shape&);
 unsigned gemv_error_flags();
 unsigned gemv_mma_error_flags();
@@ -17,12 +17,15 @@ cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const
                             float*, cudaStream_t);
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
                         void*, cudaStream_t);
+
 cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
                            uint16_t*, cudaStream_t);
 unsigned gemm_error_flags();
 
 // Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc.
 int gemv_kernel_choice = MBOK_GEMV_AUTO;
+// Process-wide promise that GEMV weights are not written by preceding work.
+bool gemv_weights_static = false;
 
 // One decode GEMV call: the lookup-table kernel once per vector, or the
 // tensor-core kernel over the whole batch.
@@ -35,7 +38,8 @@ cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shap
   const size_t xbytes = x_f32 ? 4 : 2;
   for (int b = 0; b < batch; ++b) {
     const void* xb = static_cast<const char*>(x) + size_t(b) * s.N * xbytes;
-    const cudaError_t e = launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream);
+    const cudaError_t e = launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream,
+                                          gemv_weights_static);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -150,6 +154,12 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
     return MBOK_ERR_WORKSPACE;
   return from_cuda(launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32,
                                batch, y, workspace, as_stream(stream)));
+}
+
+int mbok_gemv_set_static_weights(int on) {
+  if (on != 0 && on != 1) return MBOK_ERR_INVALID_ARG;
+  gemv_weights_static = on == 1;
+  return MBOK_OK;
 }
 
 int mbok_gemv_set_kernel(int kernel) {

@@ -68,6 +68,7 @@ struct GemvParams {
   unsigned* counter;   // [cps]
   Shape s;
   int nslab, cps;
+  int weights_static;  // bits and scales may be read before the grid dependency wait
 };
 
 // ---------------------------------------------------------------------------
@@ -267,20 +268,33 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   const int first = o_begin + warp;
   const int n_mine = first < o_end ? (o_end - first + kGemvWarps - 1) / kGemvWarps : 0;
 
-  // Before the dependency wait: only L2 prefetches of this warp's first octets.
+  // Before the dependency wait: L2 prefetches of this warp's first octets,
+  // and with static weights (the caller guarantees that nothing running
+  // before this launch writes them) the first octets' copies into shared
+  // memory as well.
   for (int t = 0; t < kPrefetchOctets && t < n_mine; ++t)
     prefetch_octet<K>(p, slab, units, groups, first + t * kGemvWarps, lane);
+  if (p.weights_static) {
+#pragma unroll
+    for (int t = 0; t < kDepth; ++t) {
+      if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
+      else cp_async_commit();   // keep one group per slot
+    }
+  }
   allow_dependents();
-  // Inputs and workspace may be written by the previous grid: wait for it.
+  // x, the workspace and (unless static) the weights may be written by the
+  // previous grid: wait for it.
   grid_dependency_wait();
 
   // x first: its load must not queue behind this warp's weight copies.
   float xv[8];
   load_x8<XF32>(p.x, q * kUnit + 8 * (warp >> 3), lane_ok, xv);
+  if (!p.weights_static) {
 #pragma unroll
-  for (int t = 0; t < kDepth; ++t) {
-    if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
-    else cp_async_commit();   // keep one group per slot
+    for (int t = 0; t < kDepth; ++t) {
+      if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
+      else cp_async_commit();   // keep one group per slot
+    }
   }
   build_tables(tab, xv, warp, lane);
   __syncthreads();
@@ -397,7 +411,7 @@ static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) 
 // y = W x for one vector; workspace as sized by gemv_lut_workspace_bytes.
 cudaError_t launch_gemv_lut(const uint8_t* packed, const uint16_t* alpha, const Shape& s,
                             const void* x, bool x_f32, float* y, void* workspace,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool weights_static) {
   const GemvPlan pl = gemv_plan(s, device_sm_count());
   GemvParams p;
   p.packed = packed;
@@ -407,6 +421,7 @@ cudaError_t launch_gemv_lut(const uint8_t* packed, const uint16_t* alpha, const 
   p.s = s;
   p.nslab = pl.nslab;
   p.cps = pl.cps;
+  p.weights_static = weights_static ? 1 : 0;
   p.partial = nullptr;
   p.counter = nullptr;
   if (pl.nslab > 1) {

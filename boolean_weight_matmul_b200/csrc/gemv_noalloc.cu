@@ -8,7 +8,7 @@ namespace mbok {
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
                         void*, cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
-                            float*, void*, cudaStream_t);
+                            float*, void*, cudaStream_t, bool);
 size_t gemv_lut_workspace_bytes(const Shape&);
 }  // namespace mbok
 

@@ -142,13 +142,29 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
               size_t workspace_bytes, void* stream);
 
 /* Kernel choice of mbok_gemv and mbok_gemv_noalloc for this process (all
- * devices, all later calls): MBOK_GEMV_AUTO (default: lookup tables for one
- * vector, tensor cores for more), MBOK_GEMV_LOOKUP (lookup tables, one
- * launch per vector) or MBOK_GEMV_TENSOR (tensor cores for any batch).  Both
- * kernels meet the accuracy stated for mbok_gemv; their results differ in
+ * devices, all later calls):
+ *   MBOK_GEMV_AUTO (default): lookup tables for one vector, tensor cores for
+ *     more;
+ *   MBOK_GEMV_LOOKUP: lookup tables (8-bit tables over 512-column slabs,
+ *     slabs combined across CTAs through the workspace), one launch per
+ *     vector;
+ *   MBOK_GEMV_TENSOR: tensor cores for any batch.
+ * Both kernels meet the accuracy stated for mbok_gemv; results differ in
  * rounding.  Not synchronised with calls in flight on other host threads.
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);
+
+/* Promise (on = 1) or withdraw (on = 0, the default) for this process that
+ * the packed bits and scales passed to later mbok_gemv / mbok_gemv_noalloc
+ * calls are never written by work that may still run on the device when the
+ * GEMV is launched -- true for inference with resident weights.  With the
+ * promise the lookup kernels copy their first weight tiles into shared
+ * memory before waiting for the preceding launch in the stream (launches
+ * overlap through programmatic dependent launch), hiding the weights' first
+ * DRAM latency behind that launch's tail.  Activations, outputs and the
+ * workspace are ordered after the preceding launch either way.  Results do
+ * not change.  Returns MBOK_ERR_INVALID_ARG for other values. */
+int mbok_gemv_set_static_weights(int on);
 
 /* mbok_gemv without a workspace argument, for callers that cannot allocate
  * device memory: code that must not call cudaMalloc after start-up (an

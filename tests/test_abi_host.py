@@ -108,3 +108,9 @@ def test_gemv_kernel_choice(L):
         pass
     with pytest.raises(mb.MbokError):
         mb.gemv_set_kernel(7)
+
+
+def test_gemv_static_weights_switch(L):
+    assert L.mbok_gemv_set_static_weights(2) == 1 and L.mbok_gemv_set_static_weights(-1) == 1
+    assert L.mbok_gemv_set_static_weights(1) == 0
+    assert L.mbok_gemv_set_static_weights(0) == 0

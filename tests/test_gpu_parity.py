@@ -288,6 +288,49 @@ def test_gemv_kernel_flip_invariance_bitwise(kernel):
             assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
 
 
+@pytest.mark.parametrize("M,N", [(4096, 4096), (300, 1536), (5120, 13824)])
+def test_gemv_static_weights_same_bits(M, N):
+    # Copying weights into shared memory before the dependency wait changes
+    # no result: bit-identical outputs, also for a chain of launches whose
+    # inputs the previous launch wrote.
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    K = 3
+    s = wl.random_signs(K, M, N, 101)
+    a = wl.alpha_decaying(K, M, N, 102)
+    x = wl.x_normal(1, N, 103)
+    p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
+    with mb.gemv_kernel(mb.GEMV_LOOKUP):
+        y0 = gemv_gpu(p, al, K, M, N, x, "bf16")
+        mb.gemv_set_static_weights(True)
+        try:
+            y1 = gemv_gpu(p, al, K, M, N, x, "bf16")
+            # chain: y of one launch (bf16) is the x of the next, no host sync between
+            xs = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+            ws = mb.zeros_workspace(K, M, N, 1)
+            ys = []
+            cur = xs
+            for _ in range(3):
+                y = torch.empty(1, M, dtype=torch.float32, device="cuda")
+                mb.gemv(p, al, K, M, N, 128, cur, mb.BF16, 1, y, ws)
+                ys.append(y)
+                if M == N:
+                    cur = (y * 0.05).to(torch.bfloat16)
+            torch.cuda.synchronize()
+        finally:
+            mb.gemv_set_static_weights(False)
+    assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
+    assert_close(y1, *O.linear(O.pack_signs(s), a, K, M, N, x, "bf16"), GEMV_REL_L2, "static weights")
+    if M == N:
+        # each link of the chain against the oracle on the activations it actually read
+        cur = x
+        for y in ys:
+            yn = y.cpu().numpy()
+            y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, cur, "bf16")
+            assert_close(yn, y_ref, E, GEMV_REL_L2, "static weights chain")
+            cur = wl.f32_to_bf16_bits((yn * np.float32(0.05)).astype(np.float32))
+
+
 def test_gemv_tensor_deterministic_and_batch_independent():
     # Same bits run to run; a vector's result does not depend on its batch
     # neighbours (columns of B never mix) among batches that use the same
