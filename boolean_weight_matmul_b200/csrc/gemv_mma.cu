@@ -20,20 +20,19 @@
 //    and added into the output accumulators (fp32 FMA), so the scales are
 //    applied exactly as the method's grouped sum states.
 //  * A CTA owns one 16-row tile (two storage octets) and all N columns.  The
-//    tile's bits and scales and the activations stream through a 4-stage
-//    shared-memory ring in column slices (1024 columns; 512 when B has 16
-//    columns): per slice, one bulk asynchronous copy per (octet, kernel) (the
-//    slice is contiguous in storage format 1), one per octet for the scales
-//    and one per activation vector, all completing on the stage's mbarrier.
-//    The 8 warps split a slice's 64-column chunks; their partial sums meet in
-//    shared memory, summed in warp order: no cross-CTA combine, no
-//    workspace, deterministic.
+//    tile's bits and scales stream through a 4-stage shared-memory ring in
+//    1024-column slices: per slice, one bulk asynchronous copy per (octet,
+//    kernel) (the slice is contiguous in storage format 1) and one per octet
+//    for the scales, completing on the stage's mbarrier.  The 8 warps split
+//    a slice's 64-column chunks; their partial sums meet in shared memory,
+//    summed in warp order: no cross-CTA combine, no workspace,
+//    deterministic.  Activations are shared by all CTAs, so they are read
+//    from global memory (L1/L2-resident), one chunk ahead of their use.
 //  * The k-index of an MMA is a permutation of the 16 columns it covers:
 //    thread (g, t) of a warp reads the halfword of row g for unit 4c + t of
 //    chunk c, and MMA j of the chunk takes bits 4j..4j+3 of it (columns
 //    16(4c+t) + 4j .. +3).  B uses the same permutation, which is simply 16
-//    consecutive activations of that unit per thread (vector rows padded by
-//    16 bytes in shared memory so these reads are conflict-free).
+//    consecutive activations of that unit per thread.
 //  * Launches use programmatic dependent launch: before waiting on the
 //    previous grid a CTA only asks L2 to prefetch its tile's bits and scales.
 //  * Every mbarrier wait is bounded (1 s); on timeout the CTA records an
@@ -53,22 +52,20 @@ constexpr unsigned long long kMmaWaitNs = 1000000000ull;
 constexpr unsigned long long kMmaDrainNs = 200000000ull;
 
 // One ring stage: a slice of kCols columns of the tile's two octets (bits of
-// every kernel, scales) and of every activation vector.  Narrower slices when
-// B has 16 columns keep the activations' share of a stage bounded.
+// every kernel, scales).  Activations are read from global memory (they are
+// shared by every CTA and stay in L1/L2), one chunk ahead of their use.
 template <int K, int NT, bool XF32>
 struct MmaGeom {
-  static constexpr int kCols = NT == 1 ? 1024 : 512;
+  static constexpr int kCols = 1024;
   static constexpr int kUnits = kCols / kUnit;
   static constexpr int kGroups = kCols / kGroup;
-  static constexpr int kXElem = XF32 ? 4 : 2;
+  static constexpr int kChunks = kCols / kChunkCols;
   static constexpr int kMaxVec = XF32 ? (8 * NT) / 3 : 8 * NT;
-  static constexpr int kXStride = kCols * kXElem + 16;          // padded: conflict-free B reads
   static constexpr int kBits = 2 * K * kUnits * 16;             // [octet][k][unit][8 rows][2 B]
   static constexpr int kAlpha = 2 * kGroups * K * 16;           // [octet][group][k][8 rows][2 B]
+  static constexpr int kStage = kBits + kAlpha;
   static constexpr int kRed = kMmaWarps * NT * 8 * 16 * 4;
-  // [bits | scales | nb activation rows]; the ring holds kMmaStages of these.
-  static constexpr int stage_bytes(int nb) { return kBits + kAlpha + nb * kXStride; }
-  static constexpr int smem_bytes(int nb) { return kMmaStages * stage_bytes(nb) + kRed; }
+  static constexpr int kSmem = kMmaStages * kStage + kRed;
 };
 
 __device__ unsigned int g_gemv_mma_error;
@@ -189,27 +186,27 @@ __device__ __forceinline__ uint32_t bf16_part(float v, int part) {
 }
 
 // The B fragment words of one chunk for column n of B: the 16 activations of
-// unit uq of the stage's slice, vector n (or n/3, part n%3, for fp32), as 8
-// bf16 pairs; zeros for unused columns.
-template <bool XF32, int XS>
-__device__ __forceinline__ void load_b(const unsigned char* xs, int nb, int n, int uq, uint32_t b[8]) {
+// unit q of vector n (or n/3, part n%3, for fp32) as 8 bf16 pairs; zeros for
+// unused columns.
+template <bool XF32>
+__device__ __forceinline__ void load_b(const GemvMmaParams& p, int n, int q, uint32_t b[8]) {
   const int vec = XF32 ? n / 3 : n;
-  if (vec >= nb) {
+  if (vec >= p.nb) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) b[i] = 0u;
     return;
   }
   if (!XF32) {
-    const uint4* src = reinterpret_cast<const uint4*>(xs + vec * XS + uq * kUnit * 2);
-    const uint4 v0 = src[0], v1 = src[1];
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + size_t(vec) * p.s.N + q * kUnit);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
     b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
     b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
   } else {
     const int part = n - 3 * vec;
-    const float4* src = reinterpret_cast<const float4*>(xs + vec * XS + uq * kUnit * 4);
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + size_t(vec) * p.s.N + q * kUnit);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 v = src[i];
+      const float4 v = __ldg(src + i);
       b[2 * i] = bf16_part(v.x, part) | (bf16_part(v.y, part) << 16);
       b[2 * i + 1] = bf16_part(v.z, part) | (bf16_part(v.w, part) << 16);
     }
@@ -220,8 +217,7 @@ __device__ __forceinline__ void load_b(const unsigned char* xs, int nb, int n, i
 // The kernel
 // ---------------------------------------------------------------------------
 
-// Thread 0: copy slice `sl` of the tile (octets o0, o0+1) and of the
-// activations into a ring stage.
+// Thread 0: copy slice `sl` of the tile (octets o0, o0+1) into a ring stage.
 template <int K, int NT, bool XF32>
 __device__ __forceinline__ void issue_slice(const GemvMmaParams& p, int o0, int n_oct, int sl, unsigned char* stage,
                                             uint64_t* full) {
@@ -232,8 +228,7 @@ __device__ __forceinline__ void issue_slice(const GemvMmaParams& p, int o0, int 
   const int ng = nu / kUnitsPerGroup;
   const uint32_t bits_bytes = uint32_t(nu) * 16;
   const uint32_t alpha_bytes = uint32_t(ng) * K * 16;
-  const uint32_t x_bytes = uint32_t(nu) * kUnit * G::kXElem;
-  mm_arrive_expect_tx(full, uint32_t(n_oct) * (K * bits_bytes + alpha_bytes) + uint32_t(p.nb) * x_bytes);
+  mm_arrive_expect_tx(full, uint32_t(n_oct) * (K * bits_bytes + alpha_bytes));
   for (int oi = 0; oi < n_oct; ++oi) {
 #pragma unroll
     for (int k = 0; k < K; ++k)
@@ -241,27 +236,206 @@ __device__ __forceinline__ void issue_slice(const GemvMmaParams& p, int o0, int 
     bulk_copy(stage + G::kBits + oi * G::kGroups * K * 16, p.alpha + alpha_offset(s, o0 + oi, u0 / kUnitsPerGroup, 0),
               alpha_bytes, full);
   }
-  const unsigned char* x = static_cast<const unsigned char*>(p.x);
-  for (int v = 0; v < p.nb; ++v)
-    bulk_copy(stage + G::kBits + G::kAlpha + v * G::kXStride,
-              x + (size_t(v) * s.N + size_t(u0) * kUnit) * G::kXElem, x_bytes, full);
+}
+
+// Whether a group's scaling is deferred by one slice (two accumulator sets)
+// or done right after its MMAs (one set, for the register-heavy variants).
+template <int K, int NT>
+struct MmaDefer {
+  static constexpr bool value = !(NT == 2 && K >= 3);
+  static constexpr int kSets = value ? 2 : 1;
+};
+
+// Per-warp accumulators.  Warp w owns group w of every 1024-column slice
+// (chunks 2w and 2w+1).  With deferral a group's MMAs accumulate into d[P]
+// (P = slice parity) and are scaled into the output accumulators one slice
+// later, so the next group's MMAs hide the latency of the MMA chain.
+template <int K, int NT>
+struct MmaAcc {
+  static constexpr int kSets = MmaDefer<K, NT>::kSets;
+  float d[kSets][K][NT][4];
+  bool have[kSets];
+  float y[NT][4];
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int q = 0; q < kSets; ++q) {
+      have[q] = false;
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d[q][k][nt][i] = 0.f;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
+  }
+
+  // y += alpha * d[P] with the group's scales at `alph` (group w of a stage).
+  template <int P>
+  __device__ __forceinline__ void flush(const unsigned char* alph, int w, int g, int n_oct, int groups_per_stage) {
+    if (!have[P]) return;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const float a0 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(alph + (w * K + k) * 16 + 2 * g)));
+      const float a1 = n_oct > 1 ? __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(
+                                       alph + ((groups_per_stage + w) * K + k) * 16 + 2 * g)))
+                                 : 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        y[nt][0] = __fmaf_rn(a0, d[P][k][nt][0], y[nt][0]);
+        y[nt][1] = __fmaf_rn(a0, d[P][k][nt][1], y[nt][1]);
+        y[nt][2] = __fmaf_rn(a1, d[P][k][nt][2], y[nt][2]);
+        y[nt][3] = __fmaf_rn(a1, d[P][k][nt][3], y[nt][3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[P][k][nt][i] = 0.f;
+      }
+    }
+    have[P] = false;
+  }
+};
+
+// Everything a slice step needs besides the accumulators.
+struct MmaCtx {
+  unsigned char* smem;
+  uint64_t* full;
+  uint64_t* empty;
+  int* s_abort;
+  int issued;          // thread 0: slices whose copies were issued
+  int o0, n_oct, n_slices, lane, warp, g, t;
+};
+
+// The activations of chunk `half` (0 or 1) of this warp's group in slice sl.
+template <int K, int NT, bool XF32>
+__device__ __forceinline__ void load_group_b(const GemvMmaParams& p, const MmaCtx& c, int sl, int half,
+                                             uint32_t b[NT][8]) {
+  using G = MmaGeom<K, NT, XF32>;
+  const int q = sl * G::kUnits + 8 * c.warp + 4 * half + c.t;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) load_b<XF32>(p, c.g + 8 * nt, q, b[nt]);
+}
+
+// Groups of slice sl (8, fewer in a ragged last slice).
+template <int K, int NT, bool XF32>
+__device__ __forceinline__ int slice_groups(const Shape& s, int sl) {
+  using G = MmaGeom<K, NT, XF32>;
+  return min(G::kGroups, s.G - sl * G::kGroups);
+}
+
+// MMAs of one chunk (16 rows x 64 columns, K kernels) into d[P].
+template <int P, int K, int NT, bool XF32>
+__device__ __forceinline__ void chunk_mmas(const GemvMmaParams& p, const unsigned char* bits, int uq, int g, int n_oct,
+                                           const uint32_t b[NT][8], MmaAcc<K, NT>& acc) {
+  using G = MmaGeom<K, NT, XF32>;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
+    const uint32_t h1 =
+        n_oct > 1 ? *reinterpret_cast<const uint16_t*>(bits + ((K + k) * G::kUnits + uq) * 16 + 2 * g) : 0u;
+    const uint32_t v0 = spread(h0), v1 = spread(h1);
+    uint32_t a[4][4];
+    a[0][0] = sign_pair<0>(v0, p.mul);  a[0][1] = sign_pair<0>(v1, p.mul);  a[0][2] = sign_pair<2>(v0, p.mul);  a[0][3] = sign_pair<2>(v1, p.mul);
+    a[1][0] = sign_pair<4>(v0, p.mul);  a[1][1] = sign_pair<4>(v1, p.mul);  a[1][2] = sign_pair<6>(v0, p.mul);  a[1][3] = sign_pair<6>(v1, p.mul);
+    a[2][0] = sign_pair<8>(v0, p.mul);  a[2][1] = sign_pair<8>(v1, p.mul);  a[2][2] = sign_pair<10>(v0, p.mul); a[2][3] = sign_pair<10>(v1, p.mul);
+    a[3][0] = sign_pair<12>(v0, p.mul); a[3][1] = sign_pair<12>(v1, p.mul); a[3][2] = sign_pair<14>(v0, p.mul); a[3][3] = sign_pair<14>(v1, p.mul);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc.d[P][k][nt], a[j], b[nt][2 * j], b[nt][2 * j + 1]);
+  }
+}
+
+// One slice: wait for its copies, run this warp's group into d[P]; with
+// deferral, scale the previous slice's group from that slice's (still held)
+// stage and release it, else scale this group and release this stage.  The
+// stage refilled at slice sl is that of slice sl - 2 (sl - 1 without
+// deferral), released by every warp one step earlier.  False if a wait gave
+// up.  b0 holds the activations of this warp's chunk 0 in slice sl; b1 is
+// filled with those of chunk 1, and b0 with the next slice's chunk 0.
+template <int P, int K, int NT, bool XF32>
+__device__ __forceinline__ bool mma_slice(const GemvMmaParams& p, MmaCtx& c, MmaAcc<K, NT>& acc, int sl,
+                                          uint32_t b0[NT][8], uint32_t b1[NT][8]) {
+  using G = MmaGeom<K, NT, XF32>;
+  constexpr bool kDefer = MmaDefer<K, NT>::value;
+  constexpr int kLag = kDefer ? 2 : 1;
+  constexpr int stage_bytes = G::kStage;
+  const int st = sl % kMmaStages;
+  const unsigned phase = unsigned(sl / kMmaStages) & 1u;
+  // Every decision below is made warp-uniform (the MMAs are warp-wide).
+  bool good = true;
+  if (c.warp == 0) {
+    if (c.lane == 0 && sl >= kLag && c.issued < c.n_slices) {
+      const int pst = (sl - kLag) % kMmaStages;
+      good = mm_wait(&c.empty[pst], unsigned((sl - kLag) / kMmaStages) & 1u, kMmaWaitNs);
+      if (good) {
+        issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, c.smem + pst * stage_bytes, &c.full[pst]);
+        ++c.issued;
+      }
+    }
+    good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+  }
+  if (good) good = *reinterpret_cast<volatile int*>(c.s_abort) == 0;
+  if (good) good = mm_wait(&c.full[st], phase, kMmaWaitNs);
+  good = __all_sync(0xffffffffu, good);
+  if (!good) {
+    if (c.lane == 0) {
+      atomicOr(&g_gemv_mma_error, 1u);
+      *reinterpret_cast<volatile int*>(c.s_abort) = 1;
+    }
+    return false;
+  }
+
+  const unsigned char* bits = c.smem + st * stage_bytes;
+  const int w = c.warp;
+  if (w < slice_groups<K, NT, XF32>(p.s, sl)) {
+    load_group_b<K, NT, XF32>(p, c, sl, 1, b1);
+    chunk_mmas<P, K, NT, XF32>(p, bits, 8 * w + c.t, c.g, c.n_oct, b0, acc);
+    if (sl + 1 < c.n_slices && w < slice_groups<K, NT, XF32>(p.s, sl + 1)) load_group_b<K, NT, XF32>(p, c, sl + 1, 0, b0);
+    chunk_mmas<P, K, NT, XF32>(p, bits, 8 * w + 4 + c.t, c.g, c.n_oct, b1, acc);
+    acc.have[P] = true;
+  }
+  if (kDefer) {
+    if (sl >= 1) {
+      const int pst = (sl - 1) % kMmaStages;
+      acc.template flush<MmaDefer<K, NT>::kSets - 1 - P>(c.smem + pst * stage_bytes + G::kBits, w, c.g, c.n_oct,
+                                                          G::kGroups);
+      __syncwarp();
+      if (c.lane == 0) mm_arrive(&c.empty[pst]);
+    }
+  } else {
+    acc.template flush<0>(bits + G::kBits, w, c.g, c.n_oct, G::kGroups);
+    __syncwarp();
+    if (c.lane == 0) mm_arrive(&c.empty[st]);
+  }
+  return true;
 }
 
 template <int K, int NT, bool XF32>
-__global__ void __launch_bounds__(kMmaThreads, NT == 1 ? 3 : 2) gemv_mma_kernel(GemvMmaParams p) {
+__global__ void __launch_bounds__(kMmaThreads, (NT == 2 && K >= 3) ? 1 : 2) gemv_mma_kernel(GemvMmaParams p) {
   using G = MmaGeom<K, NT, XF32>;
   extern __shared__ __align__(128) unsigned char smem[];
-  const int stage_bytes = G::stage_bytes(p.nb);
+  constexpr int stage_bytes = G::kStage;
   float (*red)[NT * 8][16] = reinterpret_cast<float (*)[NT * 8][16]>(smem + kMmaStages * stage_bytes);
   __shared__ __align__(8) uint64_t full[kMmaStages], empty[kMmaStages];
   __shared__ int s_abort;
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
+  MmaCtx c;
+  c.smem = smem;
+  c.full = full;
+  c.empty = empty;
+  c.s_abort = &s_abort;
+  c.issued = 0;
+  c.lane = threadIdx.x & 31;
+  c.warp = threadIdx.x >> 5;
+  c.g = c.lane >> 2;
+  c.t = c.lane & 3;
   const Shape& s = p.s;
-  const int o0 = 2 * blockIdx.x;
-  const int n_oct = (o0 + 1 < s.O) ? 2 : 1;
-  const int n_slices = (s.N + G::kCols - 1) / G::kCols;
+  c.o0 = 2 * blockIdx.x;
+  c.n_oct = (c.o0 + 1 < s.O) ? 2 : 1;
+  c.n_slices = (s.N + G::kCols - 1) / G::kCols;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMmaStages; ++i) {
@@ -272,15 +446,15 @@ __global__ void __launch_bounds__(kMmaThreads, NT == 1 ? 3 : 2) gemv_mma_kernel(
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   // Before the dependency wait: L2 prefetch of this tile's bits and scales.
-  if (warp == 1) {
-    const size_t bits_bytes = size_t(n_oct) * s.K * s.N;
-    const size_t alpha_bytes = size_t(n_oct) * s.G * s.K * kOctet * 2;
-    const uint8_t* bsrc = p.packed + unit_offset(s, o0, 0, 0);
-    const uint8_t* asrc = reinterpret_cast<const uint8_t*>(p.alpha + alpha_offset(s, o0, 0, 0));
+  if (c.warp == 1) {
+    const size_t bits_bytes = size_t(c.n_oct) * s.K * s.N;
+    const size_t alpha_bytes = size_t(c.n_oct) * s.G * s.K * kOctet * 2;
+    const uint8_t* bsrc = p.packed + unit_offset(s, c.o0, 0, 0);
+    const uint8_t* asrc = reinterpret_cast<const uint8_t*>(p.alpha + alpha_offset(s, c.o0, 0, 0));
     constexpr size_t kPiece = 16384;
-    for (size_t off = size_t(lane) * kPiece; off < bits_bytes; off += 32 * kPiece)
+    for (size_t off = size_t(c.lane) * kPiece; off < bits_bytes; off += 32 * kPiece)
       bulk_prefetch_l2(bsrc + off, uint32_t(min(kPiece, bits_bytes - off)));
-    if (lane == 31) {
+    if (c.lane == 31) {
       for (size_t off = 0; off < alpha_bytes; off += kPiece)
         bulk_prefetch_l2(asrc + off, uint32_t(min(kPiece, alpha_bytes - off)));
     }
@@ -289,121 +463,60 @@ __global__ void __launch_bounds__(kMmaThreads, NT == 1 ? 3 : 2) gemv_mma_kernel(
   grid_dependency_wait_mma();
   __syncthreads();   // barrier initialisation visible to all threads
 
-  int issued = 0;
   if (threadIdx.x == 0) {
-    for (; issued < kMmaStages && issued < n_slices; ++issued)
-      issue_slice<K, NT, XF32>(p, o0, n_oct, issued, smem + issued * stage_bytes, &full[issued]);
+    for (; c.issued < kMmaStages && c.issued < c.n_slices; ++c.issued)
+      issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, smem + c.issued * stage_bytes, &full[c.issued]);
   }
 
-  float yacc[NT][4];
-  float d[K][NT][4];
+  MmaAcc<K, NT> acc;
+  acc.init();
+  uint32_t b0[NT][8], b1[NT][8];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      yacc[nt][i] = 0.f;
-#pragma unroll
-      for (int k = 0; k < K; ++k) d[k][nt][i] = 0.f;
-    }
+    for (int i = 0; i < 8; ++i) b0[nt][i] = 0u;
+  if (c.warp < slice_groups<K, NT, XF32>(s, 0)) load_group_b<K, NT, XF32>(p, c, 0, 0, b0);
 
-  for (int sl = 0; sl < n_slices; ++sl) {
-    const int st = sl % kMmaStages;
-    const unsigned phase = unsigned(sl / kMmaStages) & 1u;
-    // Every decision below is made warp-uniform (the MMAs are warp-wide).
-    bool good = true;
-    if (warp == 0) {
-      // Refill: slice sl + stages - 1 goes into the stage slice sl - 1 used,
-      // once every warp has released it.
-      if (lane == 0 && sl >= 1 && issued < n_slices) {
-        const int pst = (sl - 1) % kMmaStages;
-        good = mm_wait(&empty[pst], unsigned((sl - 1) / kMmaStages) & 1u, kMmaWaitNs);
-        if (good) {
-          issue_slice<K, NT, XF32>(p, o0, n_oct, issued, smem + pst * stage_bytes, &full[pst]);
-          ++issued;
-        }
-      }
-      good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-    }
-    if (good) good = *reinterpret_cast<volatile int*>(&s_abort) == 0;
-    if (good) good = mm_wait(&full[st], phase, kMmaWaitNs);
-    good = __all_sync(0xffffffffu, good);
-    if (!good) {
-      if (lane == 0) {
-        atomicOr(&g_gemv_mma_error, 1u);
-        *reinterpret_cast<volatile int*>(&s_abort) = 1;
-      }
-      break;
-    }
-
-    const unsigned char* bits = smem + st * stage_bytes;
-    const unsigned char* alph = bits + G::kBits;
-    const unsigned char* xs = alph + G::kAlpha;
-    const int u0 = sl * G::kUnits;
-    const int nchunks = min(G::kUnits, s.Q - u0) / 4;
-    const int c_begin = warp * nchunks / kMmaWarps, c_end = (warp + 1) * nchunks / kMmaWarps;
-    int grp = c_begin * kChunkCols / kGroup;
-    for (int c = c_begin; c < c_end; ++c) {
-      const int uq = 4 * c + t;   // unit within the slice
-      uint32_t b[NT][8];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) load_b<XF32, G::kXStride>(xs, p.nb, g + 8 * nt, uq, b[nt]);
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
-        const uint32_t h1 = n_oct > 1 ? *reinterpret_cast<const uint16_t*>(bits + ((K + k) * G::kUnits + uq) * 16 + 2 * g)
-                                      : 0u;
-        const uint32_t v0 = spread(h0), v1 = spread(h1);
-        uint32_t a[4][4];
-        a[0][0] = sign_pair<0>(v0, p.mul);  a[0][1] = sign_pair<0>(v1, p.mul);  a[0][2] = sign_pair<2>(v0, p.mul);  a[0][3] = sign_pair<2>(v1, p.mul);
-        a[1][0] = sign_pair<4>(v0, p.mul);  a[1][1] = sign_pair<4>(v1, p.mul);  a[1][2] = sign_pair<6>(v0, p.mul);  a[1][3] = sign_pair<6>(v1, p.mul);
-        a[2][0] = sign_pair<8>(v0, p.mul);  a[2][1] = sign_pair<8>(v1, p.mul);  a[2][2] = sign_pair<10>(v0, p.mul); a[2][3] = sign_pair<10>(v1, p.mul);
-        a[3][0] = sign_pair<12>(v0, p.mul); a[3][1] = sign_pair<12>(v1, p.mul); a[3][2] = sign_pair<14>(v0, p.mul); a[3][3] = sign_pair<14>(v1, p.mul);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(d[k][nt], a[j], b[nt][2 * j], b[nt][2 * j + 1]);
-      }
-      // End of a 128-column group (or of this warp's part of the slice).
-      const int next_grp = (c + 1) * kChunkCols / kGroup;
-      if (c + 1 == c_end || next_grp != grp) {
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          const float a0 = __half2float(__ushort_as_half(
-              *reinterpret_cast<const uint16_t*>(alph + (grp * K + k) * 16 + 2 * g)));
-          const float a1 = n_oct > 1 ? __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(
-                                           alph + ((G::kGroups + grp) * K + k) * 16 + 2 * g)))
-                                     : 0.f;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            yacc[nt][0] = __fmaf_rn(a0, d[k][nt][0], yacc[nt][0]);
-            yacc[nt][1] = __fmaf_rn(a0, d[k][nt][1], yacc[nt][1]);
-            yacc[nt][2] = __fmaf_rn(a1, d[k][nt][2], yacc[nt][2]);
-            yacc[nt][3] = __fmaf_rn(a1, d[k][nt][3], yacc[nt][3]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d[k][nt][i] = 0.f;
-          }
-        }
-        grp = next_grp;
+  constexpr bool kDefer = MmaDefer<K, NT>::value;
+  int done = 0;   // slices completed
+  if (kDefer) {
+    for (int sl = 0; sl < c.n_slices; sl += 2) {
+      if (!mma_slice<0, K, NT, XF32>(p, c, acc, sl, b0, b1)) break;
+      ++done;
+      if (sl + 1 < c.n_slices) {
+        if (!mma_slice<MmaDefer<K, NT>::kSets - 1, K, NT, XF32>(p, c, acc, sl + 1, b0, b1)) break;
+        ++done;
       }
     }
-    __syncwarp();
-    if (lane == 0) mm_arrive(&empty[st]);
+    // The last slice's group is still pending; its stage is still held.
+    if (done == c.n_slices && c.n_slices >= 1) {
+      const int last = c.n_slices - 1;
+      const unsigned char* alph = smem + (last % kMmaStages) * stage_bytes + G::kBits;
+      if (last & 1) acc.template flush<MmaDefer<K, NT>::kSets - 1>(alph, c.warp, c.g, c.n_oct, G::kGroups);
+      else acc.template flush<0>(alph, c.warp, c.g, c.n_oct, G::kGroups);
+    }
+  } else {
+    for (int sl = 0; sl < c.n_slices; ++sl) {
+      if (!mma_slice<0, K, NT, XF32>(p, c, acc, sl, b0, b1)) break;
+      ++done;
+    }
   }
 
   // Partial sums of this warp: rows g, g+8, columns 8nt + 2t, 8nt + 2t + 1.
+  const int warp = c.warp, g = c.g, t = c.t;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    red[warp][8 * nt + 2 * t][g] = yacc[nt][0];
-    red[warp][8 * nt + 2 * t + 1][g] = yacc[nt][1];
-    red[warp][8 * nt + 2 * t][g + 8] = yacc[nt][2];
-    red[warp][8 * nt + 2 * t + 1][g + 8] = yacc[nt][3];
+    red[warp][8 * nt + 2 * t][g] = acc.y[nt][0];
+    red[warp][8 * nt + 2 * t + 1][g] = acc.y[nt][1];
+    red[warp][8 * nt + 2 * t][g + 8] = acc.y[nt][2];
+    red[warp][8 * nt + 2 * t + 1][g + 8] = acc.y[nt][3];
   }
   __syncthreads();
   const bool aborted = *reinterpret_cast<volatile int*>(&s_abort) != 0;
   if (aborted) {
     // Wait (bounded) for every copy this CTA issued, then leave without storing.
     if (threadIdx.x == 0) {
-      for (int sl = 0; sl < issued; ++sl)
+      for (int sl = 0; sl < c.issued; ++sl)
         mm_wait(&full[sl % kMmaStages], unsigned(sl / kMmaStages) & 1u, kMmaDrainNs);
     }
     return;
@@ -440,17 +553,16 @@ template <int K, int NT, bool XF32>
 static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
   auto fn = gemv_mma_kernel<K, NT, XF32>;
   using G = MmaGeom<K, NT, XF32>;
-  static bool attr_set = false;   // set once (for the largest batch), outside any stream capture
+  static bool attr_set = false;   // set once, outside any stream capture
   if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               G::smem_bytes(G::kMaxVec));
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((p.s.O + 1) / 2);
   cfg.blockDim = dim3(kMmaThreads);
-  cfg.dynamicSmemBytes = G::smem_bytes(p.nb);
+  cfg.dynamicSmemBytes = G::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
