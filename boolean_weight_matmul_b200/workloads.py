@@ -73,6 +73,17 @@ def alpha_decaying(K: int, M: int, N: int, seed: int) -> np.ndarray:
     return (u * decay[None, None, :]).astype(np.float16)
 
 
+def svid_scales(K: int, M: int, N: int, seed: int):
+    """Rank-1 scales: s_in fp16 [K][N] = RN16(U(0.8, 1.2)) and s_out fp16 [K][M] =
+    RN16(0.016 * 2^-(k-1) * U(0.8, 1.2)) for k=1..K (so s_out s_in^T is about
+    E|W| = 0.016 for W ~ N(0, 0.02^2), halving per kernel)."""
+    g = rng(seed)
+    s_in = g.uniform(0.8, 1.2, size=(K, N)).astype(np.float16)
+    decay = 0.016 * np.power(2.0, -np.arange(K, dtype=np.float64))
+    s_out = (g.uniform(0.8, 1.2, size=(K, M)) * decay[:, None]).astype(np.float16)
+    return s_in, s_out
+
+
 def x_normal(batch: int, N: int, seed: int, dtype: str = "bf16") -> np.ndarray:
     """[batch][N] activations ~ N(0,1).  dtype 'f32' gives float32; 'bf16'
     gives the bf16 bit patterns as uint16 (round-to-nearest-even)."""

@@ -50,6 +50,15 @@ Storage format, version 1 (the pages give none; this is the library's format):
   Scales alpha are fp16; logically [M][N/128][K], stored blocked as
       [octet o][group g][kernel k][row i in octet].
 
+Rank-1 scales (SVID form).  The technical summaries also write each kernel
+with its own rank-1 scale, W ~= sum_k B_k (.) (s_out^k s_in^k^T) (Italian 2A/2B,
+Dutch "Methodologie" 2, Spanish 2B): s_in^k has one value per column and
+s_out^k one per row, so y = sum_k s_out^k (.) (B_k (s_in^k (.) x)).  The
+oracle for that form (linear_svid) reconstructs W_rj = sum_k b_krj s_out_kr
+s_in_kj in fp64 (each product of two fp16 values is exact; the sum over k is
+rounded in fp64) and multiplies as above.  Scales are fp16, s_in [K][N] and
+s_out [K][M].
+
 Parity pins: see tests/test_oracle_pins.py (brute force in exact rational
 arithmetic, flip invariance, level count, least-squares closed form, residual
 norm identity, the XNOR/popcount identity, a hand-worked layout example, the
@@ -196,6 +205,31 @@ def linear(packed, alpha, K: int, M: int, N: int, x, x_dtype: str, rows=None):
     y = xf @ W.T
     E = np.abs(xf) @ np.abs(W).T
     return y, E
+
+
+# --------------------------------------------------------------------------
+# Rank-1 (SVID) scales
+# --------------------------------------------------------------------------
+
+def reconstruct_svid_rows(packed, s_in, s_out, K: int, M: int, N: int, rows) -> np.ndarray:
+    """fp64 W[rows, :] with W_rj = sum_k b_{k,r,j} * s_out[k][r] * s_in[k][j]."""
+    rows = np.asarray(rows, dtype=np.int64)
+    b = unpack_rows(packed, K, M, N, rows).astype(np.float64)                  # [K][R][N]
+    si = np.asarray(s_in, dtype=np.float16).reshape(K, N).astype(np.float64)    # [K][N]
+    so = np.asarray(s_out, dtype=np.float16).reshape(K, M).astype(np.float64)   # [K][M]
+    W = np.zeros((len(rows), N), dtype=np.float64)
+    for k in range(K):
+        W += (so[k, rows][:, None] * si[k][None, :]) * b[k]
+    return W
+
+
+def linear_svid(packed, s_in, s_out, K: int, M: int, N: int, x, x_dtype: str, rows=None):
+    """y[b][r] = sum_j W_rj x[b][j] and E[b][r] = sum_j |W_rj x[b][j]| in fp64 for
+    the rank-1-scaled kernels W = sum_k B_k (.) (s_out^k s_in^k^T)."""
+    rows = np.arange(M) if rows is None else np.asarray(rows, dtype=np.int64)
+    W = reconstruct_svid_rows(packed, s_in, s_out, K, M, N, rows)
+    xf = as_f64(x, x_dtype).reshape(-1, N)
+    return xf @ W.T, np.abs(xf) @ np.abs(W).T
 
 
 # --------------------------------------------------------------------------

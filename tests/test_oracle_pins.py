@@ -127,6 +127,88 @@ def test_flip_invariance_bitwise():
         assert np.array_equal(y0, y1)
 
 
+# --------------------------------------------------------------------------
+# Rank-1 (SVID) scales: W = sum_k B_k (.) (s_out^k s_in^k^T)
+# (Italian 2A/2B, Dutch "Methodologie" 2, Spanish 2B)
+# --------------------------------------------------------------------------
+
+def _svid_case(K, M, N, seed):
+    s = wl.random_signs(K, M, N, seed, p_zero=0.05)
+    s_in, s_out = wl.svid_scales(K, M, N, seed + 1)
+    x = wl.x_normal(2, N, seed + 2, "f32")
+    return s, s_in, s_out, x
+
+
+@pytest.mark.parametrize("K", [1, 2, 3])
+def test_svid_brute_force_exact_rational(K):
+    # y_r = sum_j (sum_k b_krj s_out_kr s_in_kj) x_j in exact rational arithmetic.
+    M, N = 3, 128
+    s, s_in, s_out, x = _svid_case(K, M, N, 400 + K)
+    y, E = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "f32")
+    for b in range(2):
+        xf = [Fraction(float(v)) for v in x[b]]
+        for r in range(M):
+            acc = Fraction(0)
+            for j in range(N):
+                w = sum(Fraction(float(s_out[k, r])) * Fraction(float(s_in[k, j])) * (1 if s[k, r, j] >= 0 else -1)
+                        for k in range(K))
+                acc += w * xf[j]
+            assert abs(y[b, r] - float(acc)) <= 1e-14 * E[b, r] + 1e-300
+
+
+def test_svid_with_unit_input_scale_is_the_grouped_form():
+    # s_in = 1: W = sum_k s_out_k B_k, i.e. the grouped form with
+    # alpha_{k,r,g} = s_out_k[r] for every group.
+    K, M, N = 3, 11, 384
+    s, _, s_out, x = _svid_case(K, M, N, 31)
+    s_in = np.ones((K, N), dtype=np.float16)
+    y, _ = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "f32")
+    alpha = np.repeat(s_out.T[:, None, :], N // 128, axis=1)          # [M][G][K]
+    y2, _ = O.linear(O.pack_signs(s), alpha, K, M, N, x, "f32")
+    assert np.allclose(y, y2, rtol=1e-12, atol=0)
+
+
+def test_svid_unit_output_scale_scales_the_input():
+    # K = 1, s_out = 1: y = B (s_in (.) x), the grouped form with alpha = 1 on
+    # the scaled input (bf16 x times fp16 s_in is exact in fp32).
+    K, M, N = 1, 9, 256
+    s = wl.random_signs(K, M, N, 41)
+    s_in, _ = wl.svid_scales(K, M, N, 42)
+    s_out = np.ones((K, M), dtype=np.float16)
+    xb = wl.x_normal(1, N, 43, "bf16")
+    y, _ = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, xb, "bf16")
+    xs = (O.as_f64(xb, "bf16") * s_in[0].astype(np.float64)).astype(np.float32)
+    assert np.array_equal(xs.astype(np.float64), O.as_f64(xb, "bf16") * s_in[0].astype(np.float64))
+    ones = np.ones((M, N // 128, K), dtype=np.float16)
+    y2, _ = O.linear(O.pack_signs(s), ones, K, M, N, xs, "f32")
+    assert np.allclose(y, y2, rtol=1e-12, atol=0)
+
+
+def test_svid_rank1_closed_form():
+    # All bits set, K = 1: W = s_out s_in^T, so y = s_out * (s_in . x).
+    K, M, N = 1, 6, 256
+    s = np.ones((K, M, N), dtype=np.int8)
+    s_in, s_out = wl.svid_scales(K, M, N, 51)
+    x = wl.x_normal(1, N, 52, "f32")
+    y, _ = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "f32")
+    dot = float(np.dot(s_in[0].astype(np.float64), x[0].astype(np.float64)))
+    assert np.allclose(y[0], s_out[0].astype(np.float64) * dot, rtol=1e-12, atol=0)
+
+
+def test_svid_flip_invariance_bitwise():
+    # Flipping B_k and negating s_out^k leaves every W entry, hence y, unchanged.
+    K, M, N = 3, 7, 256
+    s, s_in, s_out, x = _svid_case(K, M, N, 61)
+    s = np.where(s == 0, 1, s).astype(np.int8)   # a 0 entry means +1 and would not flip
+    y0, _ = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "f32")
+    for k in range(K):
+        s2, so2 = s.copy(), s_out.copy()
+        s2[k] = -s2[k]
+        so2[k] = -so2[k]
+        y1, _ = O.linear_svid(O.pack_signs(s2), s_in, so2, K, M, N, x, "f32")
+        assert np.array_equal(y0, y1)
+
+
 @pytest.mark.parametrize("K", [1, 2, 3, 4])
 def test_at_most_2_pow_K_levels(K):
     # Paper-Notes 关键设计: K kernels give 2^K weight levels.
