@@ -47,7 +47,7 @@ def args_parse():
     p.add_argument("--impl", choices=["mbok", "reference"], default="mbok")
     p.add_argument("--layers", type=int, default=48, help="distinct weight copies per step")
     p.add_argument("--no-extras", action="store_true", help="skip the secondary rows")
-    p.add_argument("--rows", default="gemm,small_batch,sweep,residual,pack",
+    p.add_argument("--rows", default="gemm,small_batch,sweep,svid,residual,pack",
                    help="comma-separated secondary rows to run")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -397,6 +397,8 @@ def run_extras(torch, mb, wl, dev, peaks, a):
         run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out)
     if "sweep" in rows:
         run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out)
+    if "svid" in rows:
+        run_svid_row(torch, mb, wl, dev, peaks, stream, g, out)
     if "residual" in rows or "pack" in rows:
         run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows)
     return out
@@ -462,6 +464,32 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
                 del gr
         del packed, al
         torch.cuda.empty_cache()
+
+
+def run_svid_row(torch, mb, wl, dev, peaks, stream, g, out):
+    # Rank-1-scaled kernels (SVID form), LLaMA-7B q_proj K=3, batch 1; distinct
+    # weight copies per graph beyond L2.
+    K, M, N = 3, 4096, 4096
+    bpl = mb.packed_bytes(K, M, N) + 2 * K * (M + N)
+    L = max(8, -(-150_000_000 // bpl))
+    packed = [torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                            device=dev, generator=g) for _ in range(L)]
+    s_in = [((torch.rand(K, N, device=dev, generator=g) * 0.4) + 0.8).to(torch.float16) for _ in range(L)]
+    s_out = [((torch.rand(K, M, device=dev, generator=g) * 0.4) + 0.8).mul(0.016).to(torch.float16) for _ in range(L)]
+    x = torch.randn(1, N, device=dev, generator=g).to(torch.bfloat16)
+    y = torch.empty(1, M, dtype=torch.float32, device=dev)
+    ws = mb.zeros_svid_workspace(K, M, N, 1, dev)
+
+    def fn():
+        for l in range(L):
+            mb.gemv_svid(packed[l], s_in[l], s_out[l], K, M, N, x, mb.BF16, 1, y, ws, stream=stream)
+    ms, gr = time_graph(torch, fn, 10, 3, stream)
+    gbs = L * bpl / (ms * 1e-3) / 1e9
+    out["gemv_svid_llama7b_q_proj_k3_4096x4096_b1"] = {
+        "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "layers": L,
+        "bytes_per_layer": bpl, "kernel": "gemv_lut8_kernel<1,false,true> (one CTA per kernel and slab)"}
+    del gr, packed, s_in, s_out
+    torch.cuda.empty_cache()
 
 
 def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
             "mbok_gemv_set_kernel": ([i], i),
             "mbok_gemv_set_static_weights": ([i], i),
+            "mbok_gemv_svid_workspace_bytes": ([i, i, i, i], sz),
+            "mbok_gemv_svid": ([vp, vp, vp, i, i, i, vp, i, i, vp, vp, sz, vp], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -157,6 +159,22 @@ def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=
                                             if isinstance(workspace, torch.Tensor) else 0)
     _check(lib().mbok_gemv(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype, batch,
                            _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv")
+
+
+def gemv_svid_workspace_bytes(K: int, M: int, N: int, batch: int = 1) -> int:
+    return int(lib().mbok_gemv_svid_workspace_bytes(K, M, N, batch))
+
+
+def zeros_svid_workspace(K: int, M: int, N: int, batch: int = 1, device="cuda") -> torch.Tensor:
+    n = max(gemv_svid_workspace_bytes(K, M, N, batch), 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gemv_svid(packed, s_in, s_out, K, M, N, x, x_dtype, batch, y, workspace, stream=None) -> None:
+    """Rank-1-scaled layer: y = sum_k s_out[k] * (B_k (s_in[k] * x)) (see include/mbok.h)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mbok_gemv_svid(_ptr(packed), _ptr(s_in), _ptr(s_out), K, M, N, _ptr(x), x_dtype, batch,
+                                _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv_svid")
 
 
 def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=None) -> None:

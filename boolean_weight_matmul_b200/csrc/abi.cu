@@ -11,6 +11,9 @@ cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __hal
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t, bool);
 size_t gemv_lut_workspace_bytes(const Shape&);
+size_t gemv_svid_workspace_bytes(const Shape&);
+cudaError_t launch_gemv_svid(const uint8_t*, const uint16_t*, const uint16_t*, const Shape&, const void*, bool,
+                             float*, void*, cudaStream_t, bool);
 unsigned gemv_error_flags();
 unsigned gemv_mma_error_flags();
 cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int,
@@ -165,6 +168,37 @@ int mbok_gemv_set_static_weights(int on) {
 int mbok_gemv_set_kernel(int kernel) {
   if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TENSOR) return MBOK_ERR_INVALID_ARG;
   gemv_kernel_choice = kernel;
+  return MBOK_OK;
+}
+
+size_t mbok_gemv_svid_workspace_bytes(int K, int M, int N, int batch) {
+  if (check_shape(K, M, N) != MBOK_OK || batch < 1 || batch > MBOK_MAX_BATCH) return 0;
+  return gemv_svid_workspace_bytes(make_shape(K, M, N));
+}
+
+int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t* s_out, int K, int M, int N,
+                   const void* x, int x_dtype, int batch, float* y, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (packed == nullptr || s_in == nullptr || s_out == nullptr || x == nullptr || y == nullptr)
+    return MBOK_ERR_INVALID_ARG;
+  if (x_dtype != MBOK_F32 && x_dtype != MBOK_BF16) return MBOK_ERR_INVALID_ARG;
+  if (batch < 1 || batch > MBOK_MAX_BATCH) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(s_in, 16) || !aligned(s_out, 2) || !aligned(x, 16) || !aligned(y, 4))
+    return MBOK_ERR_ALIGN;
+  const Shape s = make_shape(K, M, N);
+  const size_t need = gemv_svid_workspace_bytes(s);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
+    return MBOK_ERR_WORKSPACE;
+  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
+    const cudaError_t e = launch_gemv_svid(reinterpret_cast<const uint8_t*>(packed), s_in, s_out, s, xb,
+                                           x_dtype == MBOK_F32, y + size_t(b) * M, workspace, as_stream(stream),
+                                           gemv_weights_static);
+    if (e != cudaSuccess) return MBOK_ERR_CUDA;
+  }
   return MBOK_OK;
 }
 

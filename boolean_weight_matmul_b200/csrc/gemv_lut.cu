@@ -61,13 +61,16 @@ struct StageGeom {
 
 struct GemvParams {
   const uint8_t* packed;
-  const uint16_t* alpha;
+  const uint16_t* alpha;   // grouped scales (grouped form)
+  const uint16_t* s_in;    // rank-1 form: fp16 [K][N]
+  const uint16_t* s_out;   // rank-1 form: fp16 [K][M]
   const void* x;
   float* y;
-  float* partial;      // [nslab][O*8]
+  float* partial;      // [nslab * nk][O*8]
   unsigned* counter;   // [cps]
   Shape s;
   int nslab, cps;
+  int nk;              // kernels handled by separate CTAs: 1 (grouped form) or K (rank-1 form)
   int weights_static;  // bits and scales may be read before the grid dependency wait
 };
 
@@ -184,6 +187,24 @@ __device__ __forceinline__ void octet_dot(const unsigned char* tab, uint32_t lan
   }
 }
 
+// One octet of K unscaled kernels (rank-1 form: the row scale comes later).
+template <int K>
+__device__ __forceinline__ void octet_sum(const unsigned char* tab, uint32_t lane4, const uint4* bits, float2 acc[4]) {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const uint4 wv = bits[k * kUnitsPerSlab];
+    const uint32_t w[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float t0 = lut(tab, __byte_perm(w[i], lane4, 0x5504));
+      const float t1 = lut(tab + 128, __byte_perm(w[i], lane4, 0x5514));
+      const float t2 = lut(tab, __byte_perm(w[i], lane4, 0x5524));
+      const float t3 = lut(tab + 128, __byte_perm(w[i], lane4, 0x5534));
+      acc[i] = __fadd2_rn(acc[i], __fadd2_rn(make_float2(t0, t2), make_float2(t1, t3)));
+    }
+  }
+}
+
 // Sum acc (8 rows) over the 32 lanes; returns, in every lane, the total of row
 // ((lane >> 2) & 7).  Fixed order, hence deterministic.
 __device__ __forceinline__ float octet_reduce(const float2 acc2[4], int lane) {
@@ -216,37 +237,43 @@ __device__ __forceinline__ float octet_reduce(const float2 acc2[4], int lane) {
 // The kernel
 // ---------------------------------------------------------------------------
 
-// Copy octet o (this warp's K x 512 columns of bits and its 4 groups x K
-// scale vectors) into stage `st`; one commit group per octet.
-template <int K>
-__device__ __forceinline__ void issue_octet(const GemvParams& p, int slab, int units, int groups, int o,
+// Copy octet o (this warp's K x 512 columns of bits of kernels kb..kb+K-1
+// and, in the grouped form, its 4 groups x K scale vectors) into stage `st`;
+// one commit group per octet.
+template <int K, bool SV>
+__device__ __forceinline__ void issue_octet(const GemvParams& p, int slab, int units, int groups, int o, int kb,
                                             unsigned char* st, int lane) {
   using G = StageGeom<K>;
   if (lane < units) {
 #pragma unroll
     for (int k = 0; k < K; ++k)
       cp_async16(st + k * kUnitsPerSlab * 16 + lane * 16,
-                 p.packed + unit_offset(p.s, o, k, slab * kUnitsPerSlab + lane));
+                 p.packed + unit_offset(p.s, o, kb + k, slab * kUnitsPerSlab + lane));
   }
-  if (lane < groups * K)
+  if (!SV && lane < groups * K)
     cp_async16(st + G::kBits + lane * 16, p.alpha + alpha_offset(p.s, o, slab * kGroupsPerSlab, 0) + lane * 8);
   cp_async_commit();
 }
 
-template <int K>
-__device__ __forceinline__ void prefetch_octet(const GemvParams& p, int slab, int units, int groups, int o,
+template <int K, bool SV>
+__device__ __forceinline__ void prefetch_octet(const GemvParams& p, int slab, int units, int groups, int o, int kb,
                                                int lane) {
   // 128-byte lines: units*16 bytes per kernel, groups*K*16 bytes of scales
-  if (lane < (units + 7) / 8 * K) {
-    const int k = lane / ((units + 7) / 8), l = lane % ((units + 7) / 8);
-    prefetch_l2(p.packed + unit_offset(p.s, o, k, slab * kUnitsPerSlab) + 128 * l);
-  } else if (lane < (units + 7) / 8 * K + (groups * K * 16 + 127) / 128) {
-    const int l = lane - (units + 7) / 8 * K;
+  const int lines = (units + 7) / 8;
+  if (lane < lines * K) {
+    const int k = lane / lines, l = lane % lines;
+    prefetch_l2(p.packed + unit_offset(p.s, o, kb + k, slab * kUnitsPerSlab) + 128 * l);
+  } else if (!SV && lane < lines * K + (groups * K * 16 + 127) / 128) {
+    const int l = lane - lines * K;
     prefetch_l2(reinterpret_cast<const uint8_t*>(p.alpha + alpha_offset(p.s, o, slab * kGroupsPerSlab, 0)) + 128 * l);
   }
 }
 
-template <int K, bool XF32>
+// SV = false: the grouped form, K kernels per CTA, scales per (kernel, row,
+// 128-column group) applied per lookup pair.  SV = true: the rank-1 form,
+// one kernel kk per CTA (K = 1 here; p.nk CTAs per slab), the tables built
+// from s_in^kk (.) x and each row's total scaled by s_out^kk[row].
+template <int K, bool XF32, bool SV>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p) {
   using G = StageGeom<K>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -254,7 +281,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   __shared__ int s_flag;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int slab = blockIdx.x % p.nslab, c = blockIdx.x / p.nslab;
+  const int nvs = SV ? p.nslab * p.nk : p.nslab;   // (slab, kernel) CTAs per row range
+  const int vs = blockIdx.x % nvs, c = blockIdx.x / nvs;
+  const int slab = SV ? vs % p.nslab : vs;
+  const int kk = SV ? vs / p.nslab : 0;
   const int o_begin = int((long long)c * p.s.O / p.cps);
   const int o_end = int((long long)(c + 1) * p.s.O / p.cps);
   const int units = min(kUnitsPerSlab, p.s.Q - slab * kUnitsPerSlab);
@@ -264,7 +294,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   const uint32_t lane4 = 4u * lane;
   const int Mpad = p.s.O * kOctet;
   unsigned char* ring = smem + kLutBytes + warp * kDepth * G::kBytes;
-  // this warp's octets: o_begin + warp + 8t, t = 0 .. n_mine-1
+  // this warp's octets: o_begin + warp + 16t, t = 0 .. n_mine-1
   const int first = o_begin + warp;
   const int n_mine = first < o_end ? (o_end - first + kGemvWarps - 1) / kGemvWarps : 0;
 
@@ -273,11 +303,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   // before this launch writes them) the first octets' copies into shared
   // memory as well.
   for (int t = 0; t < kPrefetchOctets && t < n_mine; ++t)
-    prefetch_octet<K>(p, slab, units, groups, first + t * kGemvWarps, lane);
+    prefetch_octet<K, SV>(p, slab, units, groups, first + t * kGemvWarps, kk, lane);
   if (p.weights_static) {
 #pragma unroll
     for (int t = 0; t < kDepth; ++t) {
-      if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
+      if (t < n_mine) issue_octet<K, SV>(p, slab, units, groups, first + t * kGemvWarps, kk, ring + t * G::kBytes, lane);
       else cp_async_commit();   // keep one group per slot
     }
   }
@@ -288,11 +318,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
 
   // x first: its load must not queue behind this warp's weight copies.
   float xv[8];
-  load_x8<XF32>(p.x, q * kUnit + 8 * (warp >> 3), lane_ok, xv);
+  const int col0 = q * kUnit + 8 * (warp >> 3);
+  load_x8<XF32>(p.x, col0, lane_ok, xv);
+  if (SV && lane_ok) {
+    // rank-1 form: the kernel's input scale, applied before the tables
+    const uint4 sv = *reinterpret_cast<const uint4*>(p.s_in + size_t(kk) * p.s.N + col0);
+    const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = half2_bits_to_float2(w[e]);
+      xv[2 * e] *= f.x;
+      xv[2 * e + 1] *= f.y;
+    }
+  }
   if (!p.weights_static) {
 #pragma unroll
     for (int t = 0; t < kDepth; ++t) {
-      if (t < n_mine) issue_octet<K>(p, slab, units, groups, first + t * kGemvWarps, ring + t * G::kBytes, lane);
+      if (t < n_mine) issue_octet<K, SV>(p, slab, units, groups, first + t * kGemvWarps, kk, ring + t * G::kBytes, lane);
       else cp_async_commit();   // keep one group per slot
     }
   }
@@ -308,42 +350,47 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
     for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
     if (lane_ok) {
       const uint4* bits = reinterpret_cast<const uint4*>(st) + lane;
-      const uint4* al = reinterpret_cast<const uint4*>(st + G::kBits) + (lane / kUnitsPerGroup) * K;
-      octet_dot<K>(tab, lane4, bits, al, acc);
+      if (SV) {
+        octet_sum<K>(tab, lane4, bits, acc);
+      } else {
+        const uint4* al = reinterpret_cast<const uint4*>(st + G::kBits) + (lane / kUnitsPerGroup) * K;
+        octet_dot<K>(tab, lane4, bits, al, acc);
+      }
     }
     __syncwarp();                  // all lanes are done reading the slot
     if (t + kDepth < n_mine)
-      issue_octet<K>(p, slab, units, groups, first + (t + kDepth) * kGemvWarps, st, lane);
+      issue_octet<K, SV>(p, slab, units, groups, first + (t + kDepth) * kGemvWarps, kk, st, lane);
     else
       cp_async_commit();
-    const float total = octet_reduce(acc, lane);
+    float total = octet_reduce(acc, lane);
     const int o = first + t * kGemvWarps;
     const int row = o * kOctet + ((lane >> 2) & 7);
     if ((lane & 3) == 0) {
-      if (p.nslab == 1) {
+      if (SV) total = row < p.s.M ? total * __half2float(__ushort_as_half(p.s_out[size_t(kk) * p.s.M + row])) : 0.f;
+      if (nvs == 1) {
         if (row < p.s.M) p.y[row] = total;
       } else {
-        __stcg(p.partial + size_t(slab) * Mpad + row, total);
+        __stcg(p.partial + size_t(vs) * Mpad + row, total);
       }
     }
   }
   cp_async_wait<0>();
-  if (p.nslab == 1) return;
+  if (nvs == 1) return;
 
-  // Cross-slab combination: one release/acquire arrival per CTA; the last
-  // CTA of the row range adds the slabs' partials in slab order.
+  // Cross-CTA combination: one release/acquire arrival per CTA; the last
+  // CTA of the row range adds the partials in (kernel, slab) order.
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned prev = atomic_add_acq_rel(&p.counter[c], 1u);
-    s_flag = (prev == unsigned(p.nslab - 1));
-    if (s_flag) p.counter[c] = 0u;  // every slab of this row range has arrived
+    s_flag = (prev == unsigned(nvs - 1));
+    if (s_flag) p.counter[c] = 0u;  // every CTA of this row range has arrived
   }
   __syncthreads();
   if (!s_flag) return;
   const int r_end = min(o_end * kOctet, p.s.M);
   for (int r = o_begin * kOctet + threadIdx.x; r < r_end; r += blockDim.x) {
     float sum = 0.f;
-    for (int t = 0; t < p.nslab; ++t) sum += __ldcg(p.partial + size_t(t) * Mpad + r);
+    for (int t = 0; t < nvs; ++t) sum += __ldcg(p.partial + size_t(t) * Mpad + r);
     p.y[r] = sum;
   }
 }
@@ -356,10 +403,12 @@ struct GemvPlan {
   int nslab, cps;
 };
 
-inline GemvPlan gemv_plan(const Shape& s, int sm_count) {
+// nk = kernels given their own CTAs (1 in the grouped form, K in the rank-1
+// form): nslab * nk CTAs per row range.
+inline GemvPlan gemv_plan(const Shape& s, int sm_count, int nk) {
   GemvPlan pl;
   pl.nslab = (s.N + kSlabCols - 1) / kSlabCols;
-  int cps = sm_count / pl.nslab;
+  int cps = sm_count / (pl.nslab * nk);
   if (cps < 1) cps = 1;
   if (cps > s.O) cps = s.O;
   if (cps > int(kMaxCps)) cps = int(kMaxCps);
@@ -368,23 +417,25 @@ inline GemvPlan gemv_plan(const Shape& s, int sm_count) {
 }
 
 // Workspace: the first kCounterBytes hold one arrival counter per row range
-// (at most kMaxCps ranges); calls leave them at zero.  Per-slab partial sums
+// (at most kMaxCps ranges); calls leave them at zero.  Per-CTA partial sums
 // follow.  The counter block has a fixed size so that calls of any shape can
 // share one workspace.
-size_t gemv_lut_workspace_bytes(const Shape& s) {
-  const size_t nslab = (s.N + kSlabCols - 1) / kSlabCols;
-  if (nslab <= 1) return 0;
-  return kCounterBytes + nslab * size_t(s.O) * kOctet * sizeof(float);
+static size_t workspace_bytes_for(const Shape& s, int nk) {
+  const size_t nvs = size_t((s.N + kSlabCols - 1) / kSlabCols) * nk;
+  if (nvs <= 1) return 0;
+  return kCounterBytes + nvs * size_t(s.O) * kOctet * sizeof(float);
 }
+size_t gemv_lut_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, 1); }
+size_t gemv_svid_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, s.K); }
 
 // This kernel has no spin-waits (cp.async groups complete by themselves), so
 // it never records a device error flag.
 unsigned gemv_error_flags() { return 0u; }
 
-template <int K, bool XF32>
+template <int K, bool XF32, bool SV>
 static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) {
   using G = StageGeom<K>;
-  auto fn = gemv_lut8_kernel<K, XF32>;
+  auto fn = gemv_lut8_kernel<K, XF32, SV>;
   static bool attr_set = false;   // set once, outside any stream capture
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
@@ -408,37 +459,59 @@ static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
-// y = W x for one vector; workspace as sized by gemv_lut_workspace_bytes.
-cudaError_t launch_gemv_lut(const uint8_t* packed, const uint16_t* alpha, const Shape& s,
-                            const void* x, bool x_f32, float* y, void* workspace,
-                            cudaStream_t stream, bool weights_static) {
-  const GemvPlan pl = gemv_plan(s, device_sm_count());
+static GemvParams make_params(const uint8_t* packed, const Shape& s, const void* x, float* y, void* workspace,
+                              bool weights_static, int nk) {
+  const GemvPlan pl = gemv_plan(s, device_sm_count(), nk);
   GemvParams p;
   p.packed = packed;
-  p.alpha = alpha;
+  p.alpha = nullptr;
+  p.s_in = nullptr;
+  p.s_out = nullptr;
   p.x = x;
   p.y = y;
   p.s = s;
   p.nslab = pl.nslab;
   p.cps = pl.cps;
+  p.nk = nk;
   p.weights_static = weights_static ? 1 : 0;
   p.partial = nullptr;
   p.counter = nullptr;
-  if (pl.nslab > 1) {
+  if (pl.nslab * nk > 1) {
     p.counter = static_cast<unsigned*>(workspace);
     p.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
   }
-  const int grid = pl.nslab * pl.cps;
+  return p;
+}
+
+// y = W x for one vector; workspace as sized by gemv_lut_workspace_bytes.
+cudaError_t launch_gemv_lut(const uint8_t* packed, const uint16_t* alpha, const Shape& s,
+                            const void* x, bool x_f32, float* y, void* workspace,
+                            cudaStream_t stream, bool weights_static) {
+  GemvParams p = make_params(packed, s, x, y, workspace, weights_static, 1);
+  p.alpha = alpha;
+  const int grid = p.nslab * p.cps;
   switch (s.K * 2 + (x_f32 ? 1 : 0)) {
-    case 2: return launch_k<1, false>(p, grid, stream);
-    case 3: return launch_k<1, true>(p, grid, stream);
-    case 4: return launch_k<2, false>(p, grid, stream);
-    case 5: return launch_k<2, true>(p, grid, stream);
-    case 6: return launch_k<3, false>(p, grid, stream);
-    case 7: return launch_k<3, true>(p, grid, stream);
-    case 8: return launch_k<4, false>(p, grid, stream);
-    default: return launch_k<4, true>(p, grid, stream);
+    case 2: return launch_k<1, false, false>(p, grid, stream);
+    case 3: return launch_k<1, true, false>(p, grid, stream);
+    case 4: return launch_k<2, false, false>(p, grid, stream);
+    case 5: return launch_k<2, true, false>(p, grid, stream);
+    case 6: return launch_k<3, false, false>(p, grid, stream);
+    case 7: return launch_k<3, true, false>(p, grid, stream);
+    case 8: return launch_k<4, false, false>(p, grid, stream);
+    default: return launch_k<4, true, false>(p, grid, stream);
   }
+}
+
+// Rank-1 form: y = sum_k s_out^k (.) (B_k (s_in^k (.) x)) for one vector;
+// workspace as sized by gemv_svid_workspace_bytes.
+cudaError_t launch_gemv_svid(const uint8_t* packed, const uint16_t* s_in, const uint16_t* s_out, const Shape& s,
+                             const void* x, bool x_f32, float* y, void* workspace, cudaStream_t stream,
+                             bool weights_static) {
+  GemvParams p = make_params(packed, s, x, y, workspace, weights_static, s.K);
+  p.s_in = s_in;
+  p.s_out = s_out;
+  const int grid = p.nslab * p.nk * p.cps;
+  return x_f32 ? launch_k<1, true, true>(p, grid, stream) : launch_k<1, false, true>(p, grid, stream);
 }
 
 }  // namespace mbok

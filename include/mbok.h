@@ -141,6 +141,29 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
               const void* x, int x_dtype, int batch, float* y, void* workspace,
               size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace mbok_gemv_svid needs (same rules as
+ * mbok_gemv_workspace_bytes; one workspace may serve both calls if it has
+ * the larger of the two sizes). */
+size_t mbok_gemv_svid_workspace_bytes(int K, int M, int N, int batch);
+
+/* The rank-1-scaled form of the layer (Italian technical summary 2A/2B,
+ * Dutch "Methodologie" 2, Spanish 2B: each kernel carries its own rank-1
+ * scale, W = sum_k B_k (.) (s_out^k s_in^k^T)):
+ *     y[b][r] = sum_k s_out[k][r] * sum_j b_{k,r,j} * s_in[k][j] * x[b][j].
+ *   packed : the K sign matrices in layout 1 (as for mbok_gemv).
+ *   s_in   : fp16 [K][N] input scales, 16-byte aligned.
+ *   s_out  : fp16 [K][M] output scales.
+ *   x, x_dtype, batch, y, workspace, workspace_bytes, stream: as mbok_gemv
+ *            (workspace sized by mbok_gemv_svid_workspace_bytes).
+ * Each product s_in * x is formed in fp32 (exact for bf16 x), the +-1 sums
+ * come from lookup tables of those products (one launch per vector; each
+ * kernel k of a 512-column slab is its own CTA), and the row totals are
+ * scaled by s_out in fp32.  Accuracy and determinism as for mbok_gemv, with
+ * W the rank-1-scaled matrix above. */
+int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t* s_out, int K, int M, int N,
+                   const void* x, int x_dtype, int batch, float* y, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
 /* Kernel choice of mbok_gemv and mbok_gemv_noalloc for this process (all
  * devices, all later calls):
  *   MBOK_GEMV_AUTO (default): lookup tables for one vector, tensor cores for

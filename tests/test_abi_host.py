@@ -114,3 +114,17 @@ def test_gemv_static_weights_switch(L):
     assert L.mbok_gemv_set_static_weights(2) == 1 and L.mbok_gemv_set_static_weights(-1) == 1
     assert L.mbok_gemv_set_static_weights(1) == 0
     assert L.mbok_gemv_set_static_weights(0) == 0
+
+
+def test_gemv_svid_argument_errors(L):
+    g = lambda **kw: L.mbok_gemv_svid(*[kw.get(k, v) for k, v in dict(
+        packed=FAKE, s_in=FAKE, s_out=FAKE, K=3, M=64, N=1024, x=FAKE, dt=1, batch=1, y=FAKE,
+        ws=FAKE, wsb=1 << 20, stream=None).items()])
+    assert g(K=0) == 1 and g(K=5) == 1
+    assert g(M=0) == 2 and g(N=100) == 2
+    assert g(s_in=None) == 1 and g(s_out=None) == 1 and g(x=None) == 1
+    assert g(batch=0) == 1 and g(batch=17) == 1 and g(dt=5) == 1
+    assert g(s_in=FAKE + 8) == 3 and g(s_out=FAKE_ODD) == 3
+    assert g(ws=None) == 6 and g(wsb=16) == 6
+    assert L.mbok_gemv_svid_workspace_bytes(3, 4096, 4096, 1) > L.mbok_gemv_workspace_bytes(3, 4096, 4096, 1)
+    assert L.mbok_gemv_svid_workspace_bytes(1, 4096, 512, 1) == 0

@@ -8,7 +8,7 @@ import pytest
 
 from oracle import mbok_oracle as O
 from boolean_weight_matmul_b200 import workloads as wl
-from helpers import (BF16_OUT_REL, GEMV_REL_L2, alpha_blocked_gpu, assert_close, ensure_built, gemm_gpu,
+from helpers import (BF16_OUT_REL, GEMV_REL_L2, alpha_blocked_gpu, assert_close, ensure_built, gemm_gpu, x_dev,
                      gemv_gpu, packed_from_signs_gpu, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -350,6 +350,66 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
     assert np.array_equal(y0[:9].view(np.uint32), y9.view(np.uint32))
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
+
+
+# --------------------------------------------------------------------------
+# Rank-1 (SVID) scaled kernels
+# --------------------------------------------------------------------------
+
+def _svid_gpu(signs, s_in, s_out, x, x_dtype):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    K, M, N = signs.shape
+    batch = x.shape[0]
+    packed = packed_from_signs_gpu(signs) if signs.dtype == np.int8 else signs
+    si = to_dev(np.ascontiguousarray(s_in, dtype=np.float16).view(np.int16)).view(torch.float16)
+    so = to_dev(np.ascontiguousarray(s_out, dtype=np.float16).view(np.int16)).view(torch.float16)
+    xd = x_dev(x, x_dtype)
+    y = torch.empty(batch, M, dtype=torch.float32, device="cuda")
+    ws = mb.zeros_svid_workspace(K, M, N, batch)
+    mb.gemv_svid(packed, si, so, K, M, N, xd, mb.F32 if x_dtype == "f32" else mb.BF16, batch, y, ws)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+@pytest.mark.parametrize("M,N,batch", [(1, 128, 1), (13, 640, 3), (129, 1024, 1), (64, 1536, 2)])
+def test_gemv_svid_small_shapes(K, M, N, batch):
+    for x_dtype in ("f32", "bf16"):
+        s = wl.random_signs(K, M, N, 8000 + K + M, p_zero=0.05)
+        s_in, s_out = wl.svid_scales(K, M, N, 8001 + K + M)
+        x = wl.x_normal(batch, N, 8002 + K + M, x_dtype)
+        y = _svid_gpu(s, s_in, s_out, x, x_dtype)
+        y_ref, E = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, x_dtype)
+        assert_close(y, y_ref, E, GEMV_REL_L2, f"svid K={K} M={M} N={N} b={batch} {x_dtype}")
+
+
+@pytest.mark.parametrize("K,M,N,sample", [(3, 4096, 4096, None), (4, 13824, 5120, 256), (2, 4096, 11008, 256)])
+def test_gemv_svid_llama_shapes(K, M, N, sample):
+    s = wl.random_signs(K, M, N, 8100 + M)
+    s_in, s_out = wl.svid_scales(K, M, N, 8101 + M)
+    x = wl.x_normal(1, N, 8102 + M)
+    rows = None if sample is None else np.sort(np.random.default_rng(M).choice(M, sample, replace=False))
+    y = _svid_gpu(s, s_in, s_out, x, "bf16")
+    y_ref, E = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "bf16", rows=rows)
+    if rows is not None:
+        y = y[:, rows]
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"svid {M}x{N} K={K}")
+
+
+def test_gemv_svid_flip_invariance_and_determinism():
+    K, M, N = 3, 136, 1536
+    s = wl.random_signs(K, M, N, 8201)
+    s_in, s_out = wl.svid_scales(K, M, N, 8202)
+    x = wl.x_normal(1, N, 8203)
+    y0 = _svid_gpu(s, s_in, s_out, x, "bf16")
+    assert np.array_equal(y0.view(np.uint32), _svid_gpu(s, s_in, s_out, x, "bf16").view(np.uint32))
+    for k in range(K):
+        s2, so2 = s.copy(), s_out.copy()
+        s2[k] = -s2[k]
+        so2[k] = -so2[k]
+        y1 = _svid_gpu(s2, s_in, so2, x, "bf16")
+        assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
 
 
 # --------------------------------------------------------------------------
