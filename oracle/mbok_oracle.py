@@ -268,6 +268,91 @@ def residual_binarize(W: np.ndarray, K: int):
 # Tolerance
 # --------------------------------------------------------------------------
 
+# --------------------------------------------------------------------------
+# Closed-form scale refit for fixed kernels
+# --------------------------------------------------------------------------
+# Paper-Notes page, 关键设计 "缩放因子的高效优化": once the Boolean matrices
+# are fixed, the scales have a closed-form least-squares solution, and the
+# method alternates (fixed alpha -> update B, fixed B -> update alpha).  Per
+# (row r, group g) the scales minimise ||w - sum_k alpha_k b_k||^2 over the
+# group's 128 columns, i.e. solve G alpha = c with the Gram matrix
+# G_kl = sum_j b_kj b_lj (integers) and c_k = sum_j b_kj w_j.
+# Readings (listed in the design notes): c_k is summed in fp64 in column order;
+# the solution is adj(G) c / det(G) with the adjugate and determinant exact
+# integers, the numerator summed in fp64 over the kernels in order and
+# divided once, then rounded once fp64 -> fp16 (nearest even).  Kernels whose
+# signs on the group are linearly dependent on earlier ones (a zero
+# determinant, detected exactly) are left out in kernel order and get 0.
+
+def _int_det(a) -> int:
+    n = len(a)
+    if n == 0:
+        return 1
+    if n == 1:
+        return a[0][0]
+    total = 0
+    for col in range(n):
+        minor = [row[:col] + row[col + 1:] for row in a[1:]]
+        total += (-1) ** col * a[0][col] * _int_det(minor)
+    return total
+
+
+def _int_adjugate(a):
+    n = len(a)
+    if n == 1:
+        return [[1]]
+    adj = [[0] * n for _ in range(n)]
+    for i in range(n):
+        for j in range(n):
+            minor = [row[:j] + row[j + 1:] for k, row in enumerate(a) if k != i]
+            adj[j][i] = (-1) ** (i + j) * _int_det(minor)     # transpose of the cofactors
+    return adj
+
+
+def refit_alpha_group(b: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """b: int signs [K][128] (+-1), w: fp32 [128] -> fp16 [K] least-squares scales."""
+    K = b.shape[0]
+    bi = [[int(v) for v in b[k]] for k in range(K)]
+    G = [[sum(x * y for x, y in zip(bi[k], bi[l])) for l in range(K)] for k in range(K)]
+    c = []
+    for k in range(K):
+        acc = 0.0
+        for j in range(len(w)):
+            acc = acc + (float(w[j]) if bi[k][j] > 0 else -float(w[j]))
+        c.append(acc)
+    active = []
+    for k in range(K):
+        trial = active + [k]
+        if _int_det([[G[i][j] for j in trial] for i in trial]) != 0:
+            active = trial
+    out = np.zeros(K, dtype=np.float16)
+    if not active:
+        return out
+    Ga = [[G[i][j] for j in active] for i in active]
+    det = _int_det(Ga)
+    adj = _int_adjugate(Ga)
+    for a_idx, k in enumerate(active):
+        num = 0.0
+        for i_idx in range(len(active)):
+            num = num + float(adj[a_idx][i_idx]) * c[active[i_idx]]
+        out[k] = np.float16(num / float(det))
+    return out
+
+
+def refit_alpha(W: np.ndarray, packed, K: int, M: int, N: int, rows=None) -> np.ndarray:
+    """Least-squares scales for fixed kernels: fp16 [len(rows)][G][K]."""
+    W = np.asarray(W, dtype=np.float32)
+    rows = np.arange(M) if rows is None else np.asarray(rows, dtype=np.int64)
+    b = unpack_rows(packed, K, M, N, rows)
+    G = n_groups(N)
+    out = np.zeros((len(rows), G, K), dtype=np.float16)
+    for ri, r in enumerate(rows):
+        for g in range(G):
+            sl = slice(GROUP * g, GROUP * g + GROUP)
+            out[ri, g] = refit_alpha_group(b[:, ri, sl], W[r, sl])
+    return out
+
+
 def within_tolerance(y, y_ref, E, rel: float = 1e-3, abs_: float = 1e-6) -> np.ndarray:
     """Per-element bound |y - y_ref| <= rel * E + abs_ (boolean mask)."""
     y = np.asarray(y, dtype=np.float64)

@@ -375,3 +375,64 @@ def test_tolerance_sanity():
     assert O.within_tolerance(y + 0.5 * bound, y, E).all()
     assert not O.within_tolerance(y + 2.0 * bound, y, E).any()
     assert O.rel_l2(y, y) == 0.0
+
+
+# --------------------------------------------------------------------------
+# Closed-form scale refit for fixed kernels (Paper-Notes 关键设计,
+# 缩放因子的高效优化: least squares once B is fixed)
+# --------------------------------------------------------------------------
+
+def test_refit_k1_equals_the_greedy_closed_form():
+    # K = 1 with B = sign(w): the least-squares scale is mean|w|, which the
+    # greedy residual step computes (same fp64 sum, same single rounding).
+    W = wl.w_normal(5, 384, 71)
+    signs, alpha, _ = O.residual_binarize(W, 1)
+    a2 = O.refit_alpha(W, O.pack_signs(signs), 1, 5, 384)
+    assert np.array_equal(a2.view(np.uint16), alpha.view(np.uint16))
+
+
+@pytest.mark.parametrize("K", [2, 3, 4])
+def test_refit_matches_library_least_squares(K):
+    # Against numpy's lstsq on each group (a library routine): within fp16
+    # rounding of the fp64 solution, and the normal equations hold.
+    M, N = 4, 256
+    W = wl.w_normal(M, N, 80 + K)
+    signs = wl.random_signs(K, M, N, 90 + K)
+    a = O.refit_alpha(W, O.pack_signs(signs), K, M, N).astype(np.float64)
+    for r in range(M):
+        for g in range(N // 128):
+            B = signs[:, r, 128 * g:128 * g + 128].astype(np.float64).T        # [128][K]
+            B = np.where(B == 0, 1.0, B)
+            w = W[r, 128 * g:128 * g + 128].astype(np.float64)
+            ref = np.linalg.lstsq(B, w, rcond=None)[0]
+            ulp = np.abs(ref) * 2.0 ** -10 + 2.0 ** -24
+            assert np.all(np.abs(a[r, g] - ref) <= ulp)
+            assert np.all(np.abs(B.T @ (w - B @ ref)) <= 1e-12 * np.abs(B.T @ np.abs(w)).max())
+
+
+def test_refit_lowers_the_error_of_the_greedy_scales():
+    # Refitting all K scales jointly can only lower the squared error of the
+    # greedy (one kernel at a time) scales, up to the fp16 rounding.
+    K, M, N = 3, 6, 512
+    W = wl.w_normal(M, N, 95)
+    signs, alpha, _ = O.residual_binarize(W, K)
+    a2 = O.refit_alpha(W, O.pack_signs(signs), K, M, N)
+    Wg = O.reconstruct_W(O.pack_signs(signs), alpha, K, M, N)
+    Wr = O.reconstruct_W(O.pack_signs(signs), a2, K, M, N)
+    err_g = ((W.astype(np.float64) - Wg) ** 2).sum()
+    err_r = ((W.astype(np.float64) - Wr) ** 2).sum()
+    assert err_r <= err_g * (1 + 1e-3)
+
+
+def test_refit_dependent_kernel_gets_zero():
+    # A kernel equal (or opposite) to an earlier one on a group is dropped:
+    # scale 0, the earlier kernel takes the one-kernel least-squares scale.
+    N = 128
+    w = wl.w_normal(1, N, 97)[0]
+    b0 = np.where(wl.random_signs(1, 1, N, 98)[0, 0] >= 0, 1, -1).astype(np.int8)
+    b = np.stack([b0, -b0, np.where(w >= 0, 1, -1).astype(np.int8)])
+    a = O.refit_alpha_group(b, w).astype(np.float64)
+    assert a[1] == 0.0
+    B = np.stack([b[0], b[2]]).astype(np.float64).T
+    ref = np.linalg.lstsq(B, w.astype(np.float64), rcond=None)[0]
+    assert np.all(np.abs(a[[0, 2]] - ref) <= np.abs(ref) * 2.0 ** -10 + 2.0 ** -24)
