@@ -533,6 +533,10 @@ def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
                         5, 2, stream)
     out["residual_binarize_llama7b_gate_k3"] = {"ms": ms, "gbs_of_w": 2 * W.numel() * 4 / (ms * 1e-3) / 1e9}
     del gr
+    # Least-squares scale refit for the kernels just produced, same shape.
+    ms, gr = time_graph(torch, lambda: mb.refit_alpha(W, packed, K, M, N, 128, alpha, stream=stream), 5, 2, stream)
+    out["refit_alpha_llama7b_gate_k3"] = {"ms": ms, "gbs_of_w": W.numel() * 4 / (ms * 1e-3) / 1e9}
+    del gr
     # Packing of int8 signs, same shape.
     S = torch.randint(-1, 1, (K, M, N), dtype=torch.int8, device=dev, generator=g)
     ms, gr = time_graph(torch, lambda: mb.pack_bits(S, K, M, N, packed, stream=stream), 5, 2, stream)

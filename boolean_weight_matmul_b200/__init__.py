@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemv_set_static_weights": ([i], i),
             "mbok_gemv_svid_workspace_bytes": ([i, i, i, i], sz),
             "mbok_gemv_svid": ([vp, vp, vp, i, i, i, vp, i, i, vp, vp, sz, vp], i),
+            "mbok_refit_alpha": ([vp, vp, i, i, i, i, vp, vp], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -152,6 +153,12 @@ def pack_alpha(alpha_mgk, K, M, N, alpha_out, stream=None) -> None:
 def residual_binarize(W, M, N, K, group, packed, alpha, residual=None, stream=None) -> None:
     _check(lib().mbok_residual_binarize(_ptr(W), M, N, K, group, _ptr(packed), _ptr(alpha),
                                         _ptr(residual), _stream(stream)), "mbok_residual_binarize")
+
+
+def refit_alpha(W, packed, K, M, N, group, alpha_out, stream=None) -> None:
+    """Least-squares scales for fixed kernels (see include/mbok.h)."""
+    _check(lib().mbok_refit_alpha(_ptr(W), _ptr(packed), K, M, N, group, _ptr(alpha_out), _stream(stream)),
+           "mbok_refit_alpha")
 
 
 def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=None) -> None:

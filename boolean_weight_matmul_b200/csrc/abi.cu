@@ -8,6 +8,7 @@ cudaError_t launch_pack_bits(const int8_t*, const Shape&, uint8_t*, cudaStream_t
 cudaError_t launch_pack_alpha(const uint16_t*, const Shape&, uint16_t*, cudaStream_t);
 cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __half*, float*,
                                      cudaStream_t);
+cudaError_t launch_refit_alpha(const float*, const uint8_t*, const Shape&, __half*, cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t, bool);
 size_t gemv_lut_workspace_bytes(const Shape&);
@@ -137,6 +138,19 @@ int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint3
   return from_cuda(launch_residual_binarize(W, s, reinterpret_cast<uint8_t*>(packed),
                                             reinterpret_cast<__half*>(alpha), residual,
                                             as_stream(stream)));
+}
+
+int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N, int group, uint16_t* alpha,
+                     void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (W == nullptr || packed == nullptr || alpha == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(alpha, 16)) return MBOK_ERR_ALIGN;
+  const Shape s = make_shape(K, M, N);
+  if (s.O > 65535) return MBOK_ERR_SHAPE;
+  return from_cuda(launch_refit_alpha(W, reinterpret_cast<const uint8_t*>(packed), s,
+                                      reinterpret_cast<__half*>(alpha), as_stream(stream)));
 }
 
 int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,

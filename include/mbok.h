@@ -120,6 +120,24 @@ int mbok_pack_alpha(const uint16_t* alpha_mgk, int K, int M, int N, uint16_t* al
 int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint32_t* packed,
                            uint16_t* alpha, float* residual, void* stream);
 
+/* Least-squares scales for fixed kernels: the scale step of the alternating
+ * optimisation (Paper-Notes 关键设计: once the B_k are fixed the scales have a
+ * closed-form least-squares solution).  Per row r and group g the K scales
+ * minimise sum over the group's 128 columns of (W[r][j] - sum_k alpha_k b_kj)^2:
+ *     G alpha = c,  G_kl = sum_j b_kj b_lj (exact integers),
+ *     c_k = sum_j b_kj W[r][j] (fp64, column order),
+ *     alpha = adj(G) c / det(G) with exact integer adjugate and determinant,
+ *     the numerator summed in fp64 in kernel order, one division, one
+ *     rounding fp64 -> fp16 (nearest even).
+ * A kernel whose signs on the group depend linearly on earlier kernels (exact
+ * zero determinant) is left out, in kernel order, with scale 0.  Bit-exact and
+ * deterministic.
+ *   W      : fp32 [M][N] row-major (16-byte aligned).
+ *   packed : the K kernels, layout 1.
+ *   alpha  : out, layout 1, mbok_alpha_elems(K,M,N) fp16 elements (pad rows 0). */
+int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N, int group, uint16_t* alpha,
+                     void* stream);
+
 /* y[b][r] = sum_j W[r][j] * x[b][j] for b < batch (decode / small batch).
  * Evaluated as sum over groups and kernels of alpha[k][r][g] times the
  * +-1 dot product of B_k's group slice with x (Paper-Notes 关键设计: Wx as

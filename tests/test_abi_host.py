@@ -128,3 +128,11 @@ def test_gemv_svid_argument_errors(L):
     assert g(ws=None) == 6 and g(wsb=16) == 6
     assert L.mbok_gemv_svid_workspace_bytes(3, 4096, 4096, 1) > L.mbok_gemv_workspace_bytes(3, 4096, 4096, 1)
     assert L.mbok_gemv_svid_workspace_bytes(1, 4096, 512, 1) == 0
+
+
+def test_refit_argument_errors(L):
+    assert L.mbok_refit_alpha(FAKE, FAKE, 3, 64, 256, 64, FAKE, None) == 4
+    assert L.mbok_refit_alpha(None, FAKE, 3, 64, 256, 128, FAKE, None) == 1
+    assert L.mbok_refit_alpha(FAKE_ODD, FAKE, 3, 64, 256, 128, FAKE, None) == 3
+    assert L.mbok_refit_alpha(FAKE, FAKE, 0, 64, 256, 128, FAKE, None) == 1
+    assert L.mbok_refit_alpha(FAKE, FAKE, 3, 64, 200, 128, FAKE, None) == 2

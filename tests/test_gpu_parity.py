@@ -413,6 +413,64 @@ def test_gemv_svid_flip_invariance_and_determinism():
 
 
 # --------------------------------------------------------------------------
+# Closed-form scale refit (bit-exact)
+# --------------------------------------------------------------------------
+
+def _refit_gpu(W, packed, K):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    M, N = W.shape
+    out = mb.empty_alpha(K, M, N)
+    mb.refit_alpha(to_dev(W), packed, K, M, N, 128, out)
+    torch.cuda.synchronize()
+    return O.unblock_alpha(out.cpu().numpy(), K, M, N)
+
+
+@pytest.mark.parametrize("K,M,N", [(1, 13, 384), (2, 64, 256), (3, 37, 512), (4, 16, 1024)])
+def test_refit_bit_exact_random_kernels(K, M, N):
+    W = wl.w_normal(M, N, 9000 + K)
+    signs = wl.random_signs(K, M, N, 9001 + K, p_zero=0.02)
+    packed = packed_from_signs_gpu(signs)
+    got = _refit_gpu(W, packed, K)
+    want = O.refit_alpha(W, O.pack_signs(signs), K, M, N)
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+def test_refit_bit_exact_on_greedy_kernels_and_dependent_kernels():
+    # Kernels from the GPU residual binarisation; then kernel 2 replaced by
+    # kernel 0 negated on half the rows (exactly dependent: scale 0).
+    import boolean_weight_matmul_b200 as mb
+    K, M, N = 3, 40, 768
+    W = wl.w_normal(M, N, 9100)
+    packed = mb.empty_packed(K, M, N)
+    alpha = mb.empty_alpha(K, M, N)
+    mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
+    words = _words_u32(packed)
+    signs = O.unpack_bits(words, K, M, N)
+    got = _refit_gpu(W, packed, K)
+    assert np.array_equal(got.view(np.uint16), O.refit_alpha(W, words, K, M, N).view(np.uint16))
+    s2 = signs.copy()
+    s2[2, : M // 2] = -s2[0, : M // 2]
+    got2 = _refit_gpu(W, packed_from_signs_gpu(s2.astype(np.int8)), K)
+    want2 = O.refit_alpha(W, O.pack_signs(s2.astype(np.int8)), K, M, N)
+    assert np.array_equal(got2.view(np.uint16), want2.view(np.uint16))
+    assert np.all(want2[: M // 2, :, 2] == 0)
+
+
+def test_refit_llama7b_gate_sampled():
+    import boolean_weight_matmul_b200 as mb
+    K, M, N = 3, 11008, 4096
+    W = wl.w_normal(M, N, 9200)
+    packed = mb.empty_packed(K, M, N)
+    alpha = mb.empty_alpha(K, M, N)
+    mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
+    got = _refit_gpu(W, packed, K)
+    rows = np.sort(np.random.default_rng(3).choice(M, 64, replace=False))
+    want = O.refit_alpha(W, _words_u32(packed), K, M, N, rows=rows)
+    assert np.array_equal(got[rows].view(np.uint16), want.view(np.uint16))
+
+
+# --------------------------------------------------------------------------
 # Prefill GEMM
 # --------------------------------------------------------------------------
 
