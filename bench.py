@@ -521,6 +521,39 @@ def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):
     del gr, mats
     torch.cuda.empty_cache()
 
+    # The same layers with the projections that share an input fused along M:
+    # q, k, v (3 x 5120 rows) and gate, up (2 x 13824 rows) are one matrix each
+    # (storage format 1 concatenates along M by concatenating octets), so a
+    # layer is 4 launches instead of 7.  Then once more with static weights.
+    fused = (("qkv", 3 * 5120, 5120), ("o", 5120, 5120), ("gate_up", 2 * 13824, 5120), ("down", 5120, 13824))
+    mats = []
+    fused_bytes = 0
+    for _ in range(layers):
+        for (name, M, N) in fused:
+            p = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                              device=dev, generator=g)
+            al = torch.empty(mb.alpha_elems(K, M, N), dtype=torch.float16, device=dev)
+            al.copy_((torch.rand(al.shape, device=dev, generator=g) + 0.5) * 0.01)
+            mats.append((p, al, M, N))
+            fused_bytes += mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
+    ws = mb.zeros_workspace(K, 2 * 13824, 13824, 1, dev)
+    yout = {M: torch.empty(1, M, dtype=torch.float32, device=dev) for (_, M, _) in fused}
+
+    def sweep_fused():
+        for (p, al, M, N) in mats:
+            mb.gemv(p, al, K, M, N, 128, xin[N], mb.BF16, 1, yout[M], ws, stream=stream)
+    for static in (False, True):
+        mb.gemv_set_static_weights(static)
+        ms, gr = time_graph(torch, sweep_fused, 5, 2, stream)
+        mb.gemv_set_static_weights(False)
+        gbs = fused_bytes / (ms * 1e-3) / 1e9
+        out["sweep_llama13b_k4_40x4_fused_b1" + ("_static" if static else "")] = {
+            "ms_per_token": ms, "tokens_per_s": 1e3 / ms, "bytes_per_token": fused_bytes, "gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"], "launches": len(mats)}
+        del gr
+    del mats
+    torch.cuda.empty_cache()
+
 
 def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
     # Residual binarisation, LLaMA-7B gate 11008 x 4096, K=3.

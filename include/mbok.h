@@ -138,6 +138,12 @@ int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint3
 int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N, int group, uint16_t* alpha,
                      void* stream);
 
+/* Fusing projections that share an input (q/k/v, gate/up): matrices with the
+ * same K and N whose M are multiples of 8 concatenate along M by
+ * concatenating their packed bytes and their blocked scales (both are
+ * octet-major), and one mbok_gemv over the concatenation gives, row for row,
+ * exactly the results of the separate calls (tested). */
+
 /* y[b][r] = sum_j W[r][j] * x[b][j] for b < batch (decode / small batch).
  * Evaluated as sum over groups and kernels of alpha[k][r][g] times the
  * +-1 dot product of B_k's group slice with x (Paper-Notes 关键设计: Wx as

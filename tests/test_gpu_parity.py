@@ -352,6 +352,28 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
 
 
+def test_gemv_fused_projections_equal_separate_calls():
+    # Matrices with the same K and N whose M are multiples of 8 fuse along M by
+    # concatenating their packed bytes and blocked scales (octet-major storage):
+    # one call gives, row for row, the bits of the separate calls.
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    K, N = 3, 1280
+    Ms = (320, 64, 64)
+    parts = []
+    for i, M in enumerate(Ms):
+        s = wl.random_signs(K, M, N, 9300 + i)
+        a = wl.alpha_decaying(K, M, N, 9310 + i)
+        parts.append((packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), M))
+    for batch in (1, 4):
+        x = wl.x_normal(batch, N, 9320 + batch)
+        ys = [gemv_gpu(p, al, K, M, N, x, "bf16") for (p, al, M) in parts]
+        packed = torch.cat([p for (p, _, _) in parts])
+        alpha = torch.cat([al for (_, al, _) in parts])
+        y = gemv_gpu(packed, alpha, K, sum(Ms), N, x, "bf16")
+        assert np.array_equal(y.view(np.uint32), np.concatenate(ys, axis=1).view(np.uint32))
+
+
 # --------------------------------------------------------------------------
 # Rank-1 (SVID) scaled kernels
 # --------------------------------------------------------------------------
