@@ -269,6 +269,57 @@ def residual_binarize(W: np.ndarray, K: int):
 # --------------------------------------------------------------------------
 
 # --------------------------------------------------------------------------
+# Successive SVID (rank-1 scales extracted kernel by kernel)
+# --------------------------------------------------------------------------
+# Dutch technical summary, "Methodologie" 2 (Successive SVID), Italian 2A and
+# Spanish 2B: take a rank-1 approximation of the absolute values (via SVD) to
+# get the scale vectors, the signs as the Boolean matrix, and give the
+# residual to the next kernel:
+#     B_k = sign(R_{k-1}),  |R_{k-1}| ~ sigma u v^T,
+#     s_out^k = sqrt(sigma) u,  s_in^k = sqrt(sigma) v   (u, v >= 0),
+#     R_k = R_{k-1} - B_k (.) (s_out^k s_in^k^T).
+# Readings (listed in the design notes): sign(0) = +1; the top singular
+# triple of the nonnegative |R| is taken with u, v >= 0 (its Perron vectors);
+# the product is split evenly (sqrt(sigma) on each side); s_out and s_in are
+# rounded once to fp16 (nearest even) from fp64, and the residual update uses
+# those fp16 values: R <- R - b * (s_out_r * s_in_j) as one fp32 product
+# (exact: two 11-bit significands) and one fp32 subtraction.
+
+def svid_scales_of(A: np.ndarray):
+    """Rank-1 scales of a nonnegative matrix: fp16 (s_out [M], s_in [N])."""
+    U, S, Vt = np.linalg.svd(np.asarray(A, dtype=np.float64), full_matrices=False)
+    u, v, sigma = U[:, 0], Vt[0], S[0]
+    if u.sum() < 0:
+        u, v = -u, -v
+    u, v = np.abs(u), np.abs(v)      # Perron vectors of a nonnegative matrix
+    root = math.sqrt(sigma)
+    return (root * u).astype(np.float16), (root * v).astype(np.float16)
+
+
+def svid_step(R: np.ndarray, s_out: np.ndarray, s_in: np.ndarray):
+    """One update with given fp16 scales: (signs int8 [M][N], R_next fp32)."""
+    R = np.asarray(R, dtype=np.float32)
+    b = np.where(R >= 0, 1, -1).astype(np.int8)
+    prod = np.asarray(s_out, dtype=np.float16).astype(np.float32)[:, None] * \
+        np.asarray(s_in, dtype=np.float16).astype(np.float32)[None, :]
+    R_next = (R - np.where(b > 0, prod, -prod)).astype(np.float32)
+    return b, R_next
+
+
+def svid_binarize(W: np.ndarray, K: int):
+    """fp32 W [M][N] -> (signs int8 [K][M][N], s_in fp16 [K][N], s_out fp16 [K][M], R_K fp32)."""
+    R = np.asarray(W, dtype=np.float32).copy()
+    M, N = R.shape
+    signs = np.zeros((K, M, N), dtype=np.int8)
+    s_in = np.zeros((K, N), dtype=np.float16)
+    s_out = np.zeros((K, M), dtype=np.float16)
+    for k in range(K):
+        s_out[k], s_in[k] = svid_scales_of(np.abs(R.astype(np.float64)))
+        signs[k], R = svid_step(R, s_out[k], s_in[k])
+    return signs, s_in, s_out, R
+
+
+# --------------------------------------------------------------------------
 # Closed-form scale refit for fixed kernels
 # --------------------------------------------------------------------------
 # Paper-Notes page, 关键设计 "缩放因子的高效优化": once the Boolean matrices

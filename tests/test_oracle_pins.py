@@ -436,3 +436,58 @@ def test_refit_dependent_kernel_gets_zero():
     B = np.stack([b[0], b[2]]).astype(np.float64).T
     ref = np.linalg.lstsq(B, w.astype(np.float64), rcond=None)[0]
     assert np.all(np.abs(a[[0, 2]] - ref) <= np.abs(ref) * 2.0 ** -10 + 2.0 ** -24)
+
+
+# --------------------------------------------------------------------------
+# Successive SVID (Dutch "Methodologie" 2, Italian 2A, Spanish 2B)
+# --------------------------------------------------------------------------
+
+def test_svid_constant_magnitude_is_exact():
+    # |W| = c everywhere is exactly rank 1: sigma = c sqrt(MN), u, v constant,
+    # so one kernel reproduces W and leaves R_1 = 0 (c, sqrt(M), sqrt(N) chosen
+    # so the scales are exact in fp16).
+    M, N, c = 16, 256, 0.0625     # sigma = c sqrt(MN) = 4: s_out = 0.5, s_in = 0.125
+    W = (np.where(wl.random_signs(1, M, N, 5)[0] >= 0, 1.0, -1.0) * c).astype(np.float32)
+    signs, s_in, s_out, R = O.svid_binarize(W, 1)
+    assert np.all(np.abs(R) <= 1e-9)
+    assert np.array_equal(signs[0], np.where(W >= 0, 1, -1))
+    prod = s_out[0].astype(np.float64)[:, None] * s_in[0].astype(np.float64)[None, :]
+    assert np.all(prod == c)
+
+
+def test_svid_recovers_a_rank1_scaled_sign_matrix():
+    # W = b (.) (p q^T) with positive p, q: sign(W) = b and |W| = p q^T is rank 1,
+    # so the first kernel recovers W up to the fp16 rounding of the scales.
+    M, N = 24, 384
+    b = np.where(wl.random_signs(1, M, N, 6)[0] >= 0, 1.0, -1.0)
+    g = np.random.default_rng(7)
+    p, q = g.uniform(0.5, 2.0, M), g.uniform(0.01, 0.05, N)
+    W = (b * np.outer(p, q)).astype(np.float32)
+    signs, s_in, s_out, R = O.svid_binarize(W, 1)
+    assert np.array_equal(signs[0].astype(np.float64), b)
+    assert np.max(np.abs(R)) <= 2 * 2.0 ** -11 * np.max(np.abs(W))
+
+
+def test_svid_beats_the_plain_rank1_of_w():
+    # The pages' claim: sign(W) (.) rank1(|W|) approximates W better than the
+    # rank-1 approximation of W itself.
+    W = wl.w_normal(64, 512, 8).astype(np.float64)
+    _, _, _, R = O.svid_binarize(W.astype(np.float32), 1)
+    U, S, Vt = np.linalg.svd(W, full_matrices=False)
+    plain = W - S[0] * np.outer(U[:, 0], Vt[0])
+    assert np.linalg.norm(R.astype(np.float64)) < np.linalg.norm(plain)
+
+
+def test_svid_residual_shrinks_and_signs_of_zero():
+    W = wl.w_normal(32, 256, 9)
+    W[0, :5] = 0.0
+    W[1, 3] = -0.0
+    signs, _, _, R = O.svid_binarize(W, 3)
+    assert np.all(signs[0][0, :5] == 1) and signs[0][1, 3] == 1
+    norms = [np.linalg.norm(W.astype(np.float64))]
+    R = W.copy()
+    for k in range(3):
+        so, si = O.svid_scales_of(np.abs(R.astype(np.float64)))
+        _, R = O.svid_step(R, so, si)
+        norms.append(np.linalg.norm(R.astype(np.float64)))
+    assert all(a > b for a, b in zip(norms, norms[1:]))
