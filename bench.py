@@ -566,6 +566,16 @@ def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
                         5, 2, stream)
     out["residual_binarize_llama7b_gate_k3"] = {"ms": ms, "gbs_of_w": 2 * W.numel() * 4 / (ms * 1e-3) / 1e9}
     del gr
+    # Successive SVID (rank-1 scales by 6 power iterations per kernel), same shape.
+    s_in = torch.empty(K, N, dtype=torch.float16, device=dev)
+    s_out = torch.empty(K, M, dtype=torch.float16, device=dev)
+    svws = torch.empty(int(mb.lib().mbok_svid_workspace_bytes(M, N)), dtype=torch.uint8, device=dev)
+    ms, gr = time_graph(torch, lambda: mb.svid_binarize(W, M, N, K, 6, packed, s_in, s_out, R, svws, stream=stream),
+                        3, 2, stream)
+    out["svid_binarize_llama7b_gate_k3_iters6"] = {"ms": ms, "passes_over_w": K * (2 * 6 + 2) + 1,
+                                                    "gbs_of_passes": (K * (2 * 6 + 2) + 1) * W.numel() * 4
+                                                    / (ms * 1e-3) / 1e9}
+    del gr
     # Least-squares scale refit for the kernels just produced, same shape.
     ms, gr = time_graph(torch, lambda: mb.refit_alpha(W, packed, K, M, N, 128, alpha, stream=stream), 5, 2, stream)
     out["refit_alpha_llama7b_gate_k3"] = {"ms": ms, "gbs_of_w": W.numel() * 4 / (ms * 1e-3) / 1e9}

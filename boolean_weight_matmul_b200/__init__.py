@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
             "mbok_gemv_svid_workspace_bytes": ([i, i, i, i], sz),
             "mbok_gemv_svid": ([vp, vp, vp, i, i, i, vp, i, i, vp, vp, sz, vp], i),
             "mbok_refit_alpha": ([vp, vp, i, i, i, i, vp, vp], i),
+            "mbok_svid_workspace_bytes": ([i, i], sz),
+            "mbok_svid_binarize": ([vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -153,6 +155,15 @@ def pack_alpha(alpha_mgk, K, M, N, alpha_out, stream=None) -> None:
 def residual_binarize(W, M, N, K, group, packed, alpha, residual=None, stream=None) -> None:
     _check(lib().mbok_residual_binarize(_ptr(W), M, N, K, group, _ptr(packed), _ptr(alpha),
                                         _ptr(residual), _stream(stream)), "mbok_residual_binarize")
+
+
+def svid_binarize(W, M, N, K, iters, packed, s_in, s_out, residual, workspace=None, stream=None) -> None:
+    """Successive SVID (see include/mbok.h); allocates its workspace if none is given."""
+    if workspace is None:
+        workspace = torch.empty(int(lib().mbok_svid_workspace_bytes(M, N)), dtype=torch.uint8, device=W.device)
+    _check(lib().mbok_svid_binarize(_ptr(W), M, N, K, iters, _ptr(packed), _ptr(s_in), _ptr(s_out), _ptr(residual),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mbok_svid_binarize")
 
 
 def refit_alpha(W, packed, K, M, N, group, alpha_out, stream=None) -> None:

@@ -9,6 +9,9 @@ cudaError_t launch_pack_alpha(const uint16_t*, const Shape&, uint16_t*, cudaStre
 cudaError_t launch_residual_binarize(const float*, const Shape&, uint8_t*, __half*, float*,
                                      cudaStream_t);
 cudaError_t launch_refit_alpha(const float*, const uint8_t*, const Shape&, __half*, cudaStream_t);
+size_t svid_workspace_bytes(int, int);
+cudaError_t launch_svid_binarize(const float*, const Shape&, int, uint8_t*, __half*, __half*, float*, void*,
+                                 cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t, bool);
 size_t gemv_lut_workspace_bytes(const Shape&);
@@ -138,6 +141,27 @@ int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint3
   return from_cuda(launch_residual_binarize(W, s, reinterpret_cast<uint8_t*>(packed),
                                             reinterpret_cast<__half*>(alpha), residual,
                                             as_stream(stream)));
+}
+
+size_t mbok_svid_workspace_bytes(int M, int N) {
+  if (check_shape(1, M, N) != MBOK_OK) return 0;
+  return svid_workspace_bytes(M, N);
+}
+
+int mbok_svid_binarize(const float* W, int M, int N, int K, int iters, uint32_t* packed, uint16_t* s_in,
+                       uint16_t* s_out, float* residual, void* workspace, size_t workspace_bytes, void* stream) {
+  const int st = check_shape(K, M, N);
+  if (st != MBOK_OK) return st;
+  if (iters < 1 || iters > 1000) return MBOK_ERR_INVALID_ARG;
+  if (W == nullptr || packed == nullptr || s_in == nullptr || s_out == nullptr || residual == nullptr)
+    return MBOK_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(s_in, 2) || !aligned(s_out, 2) || !aligned(residual, 16))
+    return MBOK_ERR_ALIGN;
+  if (workspace == nullptr || workspace_bytes < svid_workspace_bytes(M, N) || !aligned(workspace, 16))
+    return MBOK_ERR_WORKSPACE;
+  return from_cuda(launch_svid_binarize(W, make_shape(K, M, N), iters, reinterpret_cast<uint8_t*>(packed),
+                                        reinterpret_cast<__half*>(s_in), reinterpret_cast<__half*>(s_out), residual,
+                                        workspace, as_stream(stream)));
 }
 
 int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N, int group, uint16_t* alpha,

@@ -120,6 +120,32 @@ int mbok_pack_alpha(const uint16_t* alpha_mgk, int K, int M, int N, uint16_t* al
 int mbok_residual_binarize(const float* W, int M, int N, int K, int group, uint32_t* packed,
                            uint16_t* alpha, float* residual, void* stream);
 
+/* Bytes of device workspace mbok_svid_binarize needs for an M x N matrix. */
+size_t mbok_svid_workspace_bytes(int M, int N);
+
+/* Successive SVID: K kernels with rank-1 scales extracted one after another
+ * (Dutch technical summary "Methodologie" 2, Italian 2A, Spanish 2B: the
+ * signs of the residual, a rank-1 approximation of its absolute values as
+ * the scale vectors, the residual passed on).  Starting from R = W, for
+ * k = 0..K-1:
+ *     B_k     = sign(R), sign(0) = +1,
+ *     |R| ~ sigma u v^T with u, v >= 0: the top singular pair by `iters`
+ *              power iterations from the uniform vector (u = |R| v,
+ *              v = |R|^T u / ||.||), then u = |R| v, sigma = ||u||,
+ *     s_out[k] = fp16(u / sqrt(sigma)),  s_in[k] = fp16(sqrt(sigma) v),
+ *     R       = R - b * (s_out[k][r] * s_in[k][j])  (fp32, the fp16 scales).
+ * All sums run in a fixed order, so results are deterministic.  Evaluate the
+ * result with mbok_gemv_svid.
+ *   W        : fp32 [M][N] (16-byte aligned), not modified.
+ *   iters    : power iterations per kernel, 1..1000 (6 is ample for
+ *              weight-like matrices, whose |R| has a dominant singular value).
+ *   packed   : out, layout 1.   s_in: out, fp16 [K][N].   s_out: out, fp16 [K][M].
+ *   residual : out, fp32 [M][N] = R after the K-th kernel (also the working
+ *              buffer; 16-byte aligned).
+ *   workspace: mbok_svid_workspace_bytes(M, N) bytes, 16-byte aligned. */
+int mbok_svid_binarize(const float* W, int M, int N, int K, int iters, uint32_t* packed, uint16_t* s_in,
+                       uint16_t* s_out, float* residual, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Least-squares scales for fixed kernels: the scale step of the alternating
  * optimisation (Paper-Notes 关键设计: once the B_k are fixed the scales have a
  * closed-form least-squares solution).  Per row r and group g the K scales

@@ -136,3 +136,14 @@ def test_refit_argument_errors(L):
     assert L.mbok_refit_alpha(FAKE_ODD, FAKE, 3, 64, 256, 128, FAKE, None) == 3
     assert L.mbok_refit_alpha(FAKE, FAKE, 0, 64, 256, 128, FAKE, None) == 1
     assert L.mbok_refit_alpha(FAKE, FAKE, 3, 64, 200, 128, FAKE, None) == 2
+
+
+def test_svid_binarize_argument_errors(L):
+    g = lambda **kw: L.mbok_svid_binarize(*[kw.get(k, v) for k, v in dict(
+        W=FAKE, M=64, N=256, K=3, iters=6, packed=FAKE, s_in=FAKE, s_out=FAKE, R=FAKE, ws=FAKE,
+        wsb=1 << 24, stream=None).items()])
+    assert g(K=0) == 1 and g(iters=0) == 1 and g(W=None) == 1 and g(R=None) == 1
+    assert g(N=100) == 2 and g(M=0) == 2
+    assert g(W=FAKE_ODD) == 3 and g(R=FAKE + 4) == 3
+    assert g(ws=None) == 6 and g(wsb=16) == 6
+    assert L.mbok_svid_workspace_bytes(64, 256) >= (64 + 2 * 256 + 256) * 4

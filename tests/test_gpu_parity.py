@@ -493,6 +493,77 @@ def test_refit_llama7b_gate_sampled():
 
 
 # --------------------------------------------------------------------------
+# Successive SVID: signs and residual bit-exact given the scales; scales
+# within one fp16 rounding of the SVD's
+# --------------------------------------------------------------------------
+
+def _svid_binarize_gpu(W, K, iters=6):
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    M, N = W.shape
+    packed = mb.empty_packed(K, M, N)
+    s_in = torch.empty(K, N, dtype=torch.float16, device="cuda")
+    s_out = torch.empty(K, M, dtype=torch.float16, device="cuda")
+    R = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    mb.svid_binarize(to_dev(W), M, N, K, iters, packed, s_in, s_out, R)
+    torch.cuda.synchronize()
+    return _words_u32(packed), s_in.cpu().numpy(), s_out.cpu().numpy(), R.cpu().numpy()
+
+
+def _check_svid_steps(W, K, words, s_in, s_out, R_gpu, rows=None):
+    # Replay the steps in the oracle with the GPU's fp16 scales: each kernel's
+    # signs and the final residual must match bit for bit; each scale must be
+    # within one fp16 ulp of the rank-1 SVD of |R| (which the oracle computes).
+    M, N = W.shape
+    signs = O.unpack_bits(words, K, M, N)
+    R = W.astype(np.float32)
+    for k in range(K):
+        so_ref, si_ref = O.svid_scales_of(np.abs(R.astype(np.float64)))
+        for got, ref in ((s_out[k], so_ref), (s_in[k], si_ref)):
+            ulp = np.spacing(np.abs(ref)).astype(np.float64)
+            assert np.all(np.abs(got.astype(np.float64) - ref.astype(np.float64)) <= ulp), f"kernel {k} scales"
+        b, R = O.svid_step(R, s_out[k], s_in[k])
+        assert np.array_equal(signs[k], b), f"kernel {k} signs"
+    assert np.array_equal(R_gpu.view(np.uint32), R.view(np.uint32))
+
+
+@pytest.mark.parametrize("K,M,N", [(1, 8, 128), (3, 300, 768), (4, 77, 1024), (2, 512, 2048)])
+def test_svid_binarize_stepwise(K, M, N):
+    W = wl.w_normal(M, N, 9400 + K + M)
+    words, s_in, s_out, R = _svid_binarize_gpu(W, K)
+    _check_svid_steps(W, K, words, s_in, s_out, R)
+
+
+def test_svid_binarize_exact_rank1_and_zero_residual():
+    # |W| constant: the first kernel is exact, the residual is 0, and the next
+    # kernel's scales are 0 (no NaN from the all-zero residual).
+    M, N, c = 16, 256, 0.0625
+    W = (np.where(wl.random_signs(1, M, N, 5)[0] >= 0, 1.0, -1.0) * c).astype(np.float32)
+    words, s_in, s_out, R = _svid_binarize_gpu(W, 2)
+    assert np.all(s_out[0] == 0.5) and np.all(s_in[0] == 0.125)
+    assert np.all(s_out[1] == 0) and np.all(s_in[1] == 0) and np.all(R == 0)
+
+
+def test_svid_binarize_then_gemv_matches_oracle():
+    # The kernels and scales it produces drive mbok_gemv_svid.
+    K, M, N = 3, 1024, 4096
+    W = wl.w_normal(M, N, 9500)
+    words, s_in, s_out, R = _svid_binarize_gpu(W, K)
+    _check_svid_steps(W, K, words, s_in, s_out, R)
+    x = wl.x_normal(1, N, 9501)
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    packed = to_dev(words.view(np.int32))
+    si = to_dev(s_in.view(np.int16)).view(torch.float16)
+    so = to_dev(s_out.view(np.int16)).view(torch.float16)
+    yd = torch.empty(1, M, dtype=torch.float32, device="cuda")
+    mb.gemv_svid(packed, si, so, K, M, N, x_dev(x, "bf16"), mb.BF16, 1, yd, mb.zeros_svid_workspace(K, M, N))
+    torch.cuda.synchronize()
+    y_ref, E = O.linear_svid(words, s_in, s_out, K, M, N, x, "bf16")
+    assert_close(yd.cpu().numpy(), y_ref, E, GEMV_REL_L2, "svid_binarize -> gemv_svid")
+
+
+# --------------------------------------------------------------------------
 # Prefill GEMM
 # --------------------------------------------------------------------------
 
