@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
+            "mbok_check_wait_timeout": ([ctypes.c_uint, vp], i),
             "mbok_gemv_set_kernel": ([i], i),
             "mbok_gemv_set_static_weights": ([i], i),
             "mbok_gemv_svid_workspace_bytes": ([i, i, i, i], sz),
@@ -240,6 +241,11 @@ def read_device_errors() -> int:
     f = ctypes.c_uint(0)
     _check(lib().mbok_read_device_errors(ctypes.byref(f)), "mbok_read_device_errors")
     return f.value
+
+
+def check_wait_timeout(timeout_us: int = 20000, stream=None) -> None:
+    """Run the bounded-wait self-check (see include/mbok.h)."""
+    _check(lib().mbok_check_wait_timeout(timeout_us, _stream(stream)), "mbok_check_wait_timeout")
 
 
 def dtype_code(x: torch.Tensor) -> int:

@@ -20,6 +20,7 @@ cudaError_t launch_gemv_svid(const uint8_t*, const uint16_t*, const uint16_t*, c
                              float*, void*, cudaStream_t, bool);
 unsigned gemv_error_flags();
 unsigned gemv_mma_error_flags();
+cudaError_t launch_wait_timeout_probe(unsigned, cudaStream_t);
 cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int,
                             float*, cudaStream_t);
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
@@ -238,6 +239,11 @@ int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t*
     if (e != cudaSuccess) return MBOK_ERR_CUDA;
   }
   return MBOK_OK;
+}
+
+int mbok_check_wait_timeout(unsigned timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return MBOK_ERR_INVALID_ARG;
+  return from_cuda(launch_wait_timeout_probe(timeout_us, as_stream(stream)));
 }
 
 int mbok_read_device_errors(unsigned* flags) {

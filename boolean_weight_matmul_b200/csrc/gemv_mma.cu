@@ -581,6 +581,24 @@ static cudaError_t launch_mma_nt(const GemvMmaParams& p, bool x_f32, cudaStream_
   return x_f32 ? launch_mma_k<K, 2, true>(p, stream) : launch_mma_k<K, 2, false>(p, stream);
 }
 
+// Self-check of the bounded waits: one warp waits, with the kernels' own wait
+// helper, on an mbarrier that nothing completes; when the wait gives up it
+// records the same flag a stuck copy would.
+__global__ void wait_timeout_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) mm_bar_init(&bar, 1);
+  __syncwarp();
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  __syncwarp();
+  const bool done = __all_sync(0xffffffffu, mm_wait(&bar, 0u, limit_ns));
+  if (!done && threadIdx.x == 0) atomicOr(&g_gemv_mma_error, 1u);
+}
+
+cudaError_t launch_wait_timeout_probe(unsigned timeout_us, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(1000ull * timeout_us);
+  return cudaGetLastError();
+}
+
 // Reads and clears the kernel's error flag; ~0u if the read itself failed.
 unsigned gemv_mma_error_flags() {
   unsigned v = 0;

@@ -275,6 +275,13 @@ int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int 
  * device.  Returns MBOK_ERR_CUDA if the flags cannot be read. */
 int mbok_read_device_errors(unsigned* flags);
 
+/* Self-check of the bounded waits that the pipelined kernels use: launches
+ * one warp that waits, with the same bounded-wait code, on an mbarrier that
+ * nothing completes.  After timeout_us microseconds (1..1000000) the wait
+ * gives up and records bit 2 of mbok_read_device_errors, exactly as a copy
+ * that never landed would; the context stays usable.  No fault, no hang. */
+int mbok_check_wait_timeout(unsigned timeout_us, void* stream);
+
 /* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill) on the tensor cores
  * (tcgen05, fp32 accumulation in tensor memory).  Wt is W in bf16: each fp16
  * scale is rounded to bf16 and the K signed scales of an element are summed

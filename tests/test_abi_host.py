@@ -147,3 +147,8 @@ def test_svid_binarize_argument_errors(L):
     assert g(W=FAKE_ODD) == 3 and g(R=FAKE + 4) == 3
     assert g(ws=None) == 6 and g(wsb=16) == 6
     assert L.mbok_svid_workspace_bytes(64, 256) >= (64 + 2 * 256 + 256) * 4
+
+
+def test_wait_timeout_check_argument_errors(L):
+    assert L.mbok_check_wait_timeout(0, None) == 1
+    assert L.mbok_check_wait_timeout(2000000, None) == 1

@@ -563,6 +563,18 @@ def test_svid_binarize_then_gemv_matches_oracle():
     assert_close(yd.cpu().numpy(), y_ref, E, GEMV_REL_L2, "svid_binarize -> gemv_svid")
 
 
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    # A wait that nothing completes ends after its limit with an error flag
+    # the host reads; the flag clears on read and the next call works.
+    import boolean_weight_matmul_b200 as mb
+    assert mb.read_device_errors() == 0
+    mb.check_wait_timeout(20000)
+    assert mb.read_device_errors() == 4
+    assert mb.read_device_errors() == 0
+    y, y_ref, E = _gemv_case(3, 64, 512, 2, "bf16", 9600)
+    assert_close(y, y_ref, E, GEMV_REL_L2, "after the timeout check")
+
+
 # --------------------------------------------------------------------------
 # Prefill GEMM
 # --------------------------------------------------------------------------
