@@ -50,6 +50,9 @@ def args_parse():
     p.add_argument("--rows", default="gemm,small_batch,sweep,svid,residual,pack",
                    help="comma-separated secondary rows to run")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-gemv", default=None, metavar="K,M,N,BATCH,KERNEL",
+                   help="profiling helper: run four launches of one GEMV (KERNEL 0 auto, 1 lookup, "
+                        "2 tensor) with L2 flushed between them, print nothing else, and exit")
     return p.parse_args()
 
 
@@ -587,8 +590,35 @@ def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
     del gr
 
 
+def profile_gemv(spec: str):
+    """Four launches of one GEMV on random weights (for an ncu capture)."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    mbuild.build()
+    K, M, N, batch, kern = (int(v) for v in spec.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                           device=dev, generator=g)
+    alpha = (torch.rand(mb.alpha_elems(K, M, N), device=dev, generator=g) * 0.01).to(torch.float16)
+    x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
+    y = torch.empty(batch, M, dtype=torch.float32, device=dev)
+    ws = mb.zeros_workspace(K, M, N, batch, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2
+    with mb.gemv_kernel(kern):
+        for _ in range(4):
+            flush.zero_()
+            mb.gemv(packed, alpha, K, M, N, 128, x, mb.BF16, batch, y, ws)
+    torch.cuda.synchronize()
+
+
 def main():
     a = args_parse()
+    if a.profile_gemv:
+        profile_gemv(a.profile_gemv)
+        return
     if a.impl == "reference":
         run_reference(a)
     else:
