@@ -315,6 +315,9 @@ def run_gpu(a):
         ms = replica_max_ms(ms, dist, dev)
         dist.barrier()
     value = replica_rate(L * bytes_per_layer, ms, world) / 1e9
+    # the lookup GEMV is one launch, plus one that adds the slabs' partials
+    # when N spans more than one 512-column slab
+    launches_per_gemv = 2 if N > 512 else 1
     us_per_layer = 1e3 * ms / L
     achieved = bytes_per_layer / (us_per_layer * 1e-6) / 1e9
     traffic = ncu_traffic("gemv_lut.cu", "gemv_lut8_q_proj_k3_4096x4096")
@@ -333,22 +336,39 @@ def run_gpu(a):
                     y_dev[l], ws, stream=stream)
         y_host.copy_(y_dev, non_blocking=True)
 
+    def time_e2e(replay):
+        with torch.cuda.stream(stream):
+            for _ in range(a.warmup):
+                replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(a.steps):
+                replay()
+            e1.record(stream)
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / a.steps
+        return replica_max_ms(t, dist, dev) if world > 1 else t
+
+    # Eagerly: one Python call per layer (host launch overhead included).
+    eager_ms = time_e2e(e2e_step)
+    # As a serving loop runs it: the whole step (copies and calls) captured
+    # once in a CUDA graph and replayed; the copies still run every step.
     with torch.cuda.stream(stream):
-        for _ in range(a.warmup):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(a.steps):
-            e2e_step()
-        e1.record(stream)
-    e1.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / a.steps
-    if world > 1:
-        e2e_ms = replica_max_ms(e2e_ms, dist, dev)
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(e2e_graph, stream=stream):
+        e2e_step()
+    e2e_ms = time_e2e(e2e_graph.replay)
     e2e = {"value": replica_rate(L * bytes_per_layer, e2e_ms, world) / 1e9, "unit": UNIT,
            "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
-           "ms_per_step": e2e_ms, "path": "mbok_gemv via the C ABI, pinned host x/y, copies in the timed region"}
+           "ms_per_step": e2e_ms,
+           "path": "mbok_gemv via the C ABI, pinned host x/y copied in and out every step; the step "
+                   "(copies + calls) captured once in a CUDA graph and replayed",
+           "eager": {"value": replica_rate(L * bytes_per_layer, eager_ms, world) / 1e9, "ms_per_step": eager_ms,
+                     "path": "the same step issued eagerly from Python, one call per layer"}}
+    del e2e_graph
 
     del graph
     extras = None
@@ -375,13 +395,13 @@ def run_gpu(a):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": "gemv_lut8_kernel<3,false>",
+                     "kernel": "gemv_lut8_kernel<3,false,false> + gemv_combine_kernel (one layer = both launches)",
                      "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
                      else "fallback 6.65 TB/s"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
-        "gpu_launches": a.steps * L,
+        "gpu_launches": a.steps * L * launches_per_gemv,
         "rows": extras,
     }
     print(json.dumps(line), flush=True)
@@ -432,8 +452,8 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
     # K=3, down 4096x11008 K=2), each on both GEMV kernels.  Enough distinct
     # weight copies per graph that they exceed L2 (>= 150 MB).
     shapes = (("q_proj", 3, 4096, 4096), ("gate", 3, 11008, 4096), ("down", 2, 4096, 11008))
-    kernels = (("lookup", mb.GEMV_LOOKUP, False), ("lookup_static", mb.GEMV_LOOKUP, True),
-               ("tensor", mb.GEMV_TENSOR, False))
+    kernels = (("lookup", mb.GEMV_LOOKUP, True), ("lookup_weights_after_wait", mb.GEMV_LOOKUP, False),
+               ("tensor", mb.GEMV_TENSOR, True))
     for (name, K, M, N) in shapes:
         bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
         L = max(8, -(-150_000_000 // bpl))
@@ -450,7 +470,7 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
             x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
             y = torch.empty(batch, M, dtype=torch.float32, device=dev)
             for (kname, kcode, static) in kernels:
-                if batch > 1 and (kname.endswith("static") or (name == "q_proj" and kname == "lookup")):
+                if batch > 1 and (kname.endswith("after_wait") or (name == "q_proj" and kname == "lookup")):
                     continue
 
                 def fn():
@@ -459,7 +479,7 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
                 mb.gemv_set_static_weights(static)
                 with mb.gemv_kernel(kcode):
                     ms, gr = time_graph(torch, fn, 10, 3, stream)
-                mb.gemv_set_static_weights(False)
+                mb.gemv_set_static_weights(True)
                 gbs = L * bpl / (ms * 1e-3) / 1e9
                 out[f"gemv_llama7b_{name}_k{K}_{M}x{N}_b{batch}_{kname}"] = {
                     "us_per_layer": 1e3 * ms / L, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
@@ -527,7 +547,8 @@ def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):
     # The same layers with the projections that share an input fused along M:
     # q, k, v (3 x 5120 rows) and gate, up (2 x 13824 rows) are one matrix each
     # (storage format 1 concatenates along M by concatenating octets), so a
-    # layer is 4 launches instead of 7.  Then once more with static weights.
+    # layer is 4 launches instead of 7.  Then once more with every weight
+    # read after the dependency wait.
     fused = (("qkv", 3 * 5120, 5120), ("o", 5120, 5120), ("gate_up", 2 * 13824, 5120), ("down", 5120, 13824))
     mats = []
     fused_bytes = 0
@@ -545,12 +566,12 @@ def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):
     def sweep_fused():
         for (p, al, M, N) in mats:
             mb.gemv(p, al, K, M, N, 128, xin[N], mb.BF16, 1, yout[M], ws, stream=stream)
-    for static in (False, True):
+    for static in (True, False):
         mb.gemv_set_static_weights(static)
         ms, gr = time_graph(torch, sweep_fused, 5, 2, stream)
-        mb.gemv_set_static_weights(False)
+        mb.gemv_set_static_weights(True)
         gbs = fused_bytes / (ms * 1e-3) / 1e9
-        out["sweep_llama13b_k4_40x4_fused_b1" + ("_static" if static else "")] = {
+        out["sweep_llama13b_k4_40x4_fused_b1" + ("" if static else "_weights_after_wait")] = {
             "ms_per_token": ms, "tokens_per_s": 1e3 / ms, "bytes_per_token": fused_bytes, "gbs": gbs,
             "frac_of_hbm": gbs / peaks["hbm_gbs"], "launches": len(mats)}
         del gr

@@ -32,8 +32,9 @@ unsigned gemm_error_flags();
 
 // Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc.
 int gemv_kernel_choice = MBOK_GEMV_AUTO;
-// Process-wide promise that GEMV weights are not written by preceding work.
-bool gemv_weights_static = false;
+// Process-wide: GEMV weights may be read before the grid dependency wait
+// (see mbok_gemv_set_static_weights).
+bool gemv_weights_static = true;
 
 // One decode GEMV call: the lookup-table kernel once per vector, or the
 // tensor-core kernel over the whole batch.

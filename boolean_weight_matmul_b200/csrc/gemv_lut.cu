@@ -14,25 +14,26 @@
 //    Entry e of lane L sits at byte e*256 + 128*h + 4L, so every lookup of a
 //    warp touches 32 distinct banks: one wavefront per 8 weight bits.  The
 //    address of a lookup is one byte permute: (byte << 8) | 4L.
-//  * Each warp streams its own row octets (octet o_begin + warp + 8t) from HBM
-//    into a private 3-deep shared-memory ring with 16-byte cp.async copies:
-//    per (octet, kernel) one copy per lane (512 contiguous bytes per warp),
-//    plus the octet's 4 groups x K scale vectors.  The main loop has no
-//    block-wide barrier.  Launches use programmatic dependent launch: before
-//    waiting on the previous grid the kernel only prefetches its first octets
-//    into L2 (coherent, so safe even if the previous grid wrote the weights);
-//    the shared-memory copies, the read of x and every write happen after the
-//    wait.  A chain of layers thus overlaps one launch's tail with the next
-//    launch's HBM traffic.
+//  * Each warp streams its own row octets (octet o_begin + warp + 16t) from
+//    HBM into a private 3-deep shared-memory ring with 16-byte cp.async
+//    copies: per (octet, kernel) one copy per lane (512 contiguous bytes per
+//    warp), plus the octet's 4 groups x K scale vectors.  The main loop has
+//    no block-wide barrier.  Launches use programmatic dependent launch:
+//    before waiting on the previous grid the kernel prefetches its first
+//    octets into L2 and (unless turned off, because a kernel that lets this
+//    grid start early might write the weights) starts their shared-memory
+//    copies; the read of x and every write happen after the wait.  A chain of
+//    layers thus overlaps one launch's tail with the next launch's weights.
 //  * Per (row pair, kernel) a lane does four lookups, one packed fp32x2 add
 //    and one packed fp32x2 FMA with the two rows' fp16 group scales.
 //  * The 32 lanes' partial sums of an octet's 8 rows are combined by a
 //    transposing shuffle butterfly.
-//  * A CTA covers one slab and a contiguous range of row octets; slabs are
-//    combined deterministically: the last CTA of a row range to arrive (one
-//    release/acquire atomic per CTA) sums the per-slab partials in slab order.
-//    (A thread-block-cluster reduction through distributed shared memory was
-//    measured slower here: its barriers wait for the slowest CTA.)
+//  * A CTA covers one slab and a contiguous range of row octets and stores
+//    its per-row partial sums; a second small grid (gemv_combine_kernel) adds
+//    the slabs' partials in slab order, deterministically.  Measured faster
+//    than combining inside this grid (a release/acquire counter and a reload
+//    by the last CTA of a row range) and than a thread-block-cluster
+//    reduction through distributed shared memory.
 // Tables are built exactly sign-symmetric (T[~e] == -T[e]), so flipping every
 // bit of a kernel and negating its scales reproduces y bit for bit.
 #include "mbok_common.cuh"
@@ -45,8 +46,6 @@ constexpr int kGroupsPerSlab = kSlabCols / kGroup;
 constexpr int kGemvThreads = 512;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kLutBytes = 256 * 256;            // 256 entries x (32 lanes x 2 tables x 4 B)
-constexpr size_t kMaxCps = 1024;                // max row ranges (counters) per call
-constexpr size_t kCounterBytes = kMaxCps * sizeof(unsigned);
 constexpr int kDepth = 3;                       // octets in flight per warp
 constexpr int kPrefetchOctets = 16;             // L2 prefetch ahead of the dependency wait, per warp
 
@@ -67,7 +66,6 @@ struct GemvParams {
   const void* x;
   float* y;
   float* partial;      // [nslab * nk][O*8]
-  unsigned* counter;   // [cps]
   Shape s;
   int nslab, cps;
   int nk;              // kernels handled by separate CTAs: 1 (grouped form) or K (rank-1 form)
@@ -95,12 +93,6 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
-
-__device__ __forceinline__ unsigned atomic_add_acq_rel(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 
 // ---------------------------------------------------------------------------
 // Lookup tables
@@ -278,7 +270,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   using G = StageGeom<K>;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* tab = smem;
-  __shared__ int s_flag;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nvs = SV ? p.nslab * p.nk : p.nslab;   // (slab, kernel) CTAs per row range
@@ -299,9 +290,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   const int n_mine = first < o_end ? (o_end - first + kGemvWarps - 1) / kGemvWarps : 0;
 
   // Before the dependency wait: L2 prefetches of this warp's first octets,
-  // and with static weights (the caller guarantees that nothing running
-  // before this launch writes them) the first octets' copies into shared
-  // memory as well.
+  // and unless the caller turned it off (mbok_gemv_set_static_weights) the
+  // first octets' copies into shared memory as well -- weights are not
+  // written by kernels that let this grid start early.
   for (int t = 0; t < kPrefetchOctets && t < n_mine; ++t)
     prefetch_octet<K, SV>(p, slab, units, groups, first + t * kGemvWarps, kk, lane);
   if (p.weights_static) {
@@ -375,24 +366,22 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
     }
   }
   cp_async_wait<0>();
-  if (nvs == 1) return;
+  // With several CTAs per row range the partials are combined by
+  // gemv_combine_kernel, launched right behind this grid.
+}
 
-  // Cross-CTA combination: one release/acquire arrival per CTA; the last
-  // CTA of the row range adds the partials in (kernel, slab) order.
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const unsigned prev = atomic_add_acq_rel(&p.counter[c], 1u);
-    s_flag = (prev == unsigned(nvs - 1));
-    if (s_flag) p.counter[c] = 0u;  // every CTA of this row range has arrived
-  }
-  __syncthreads();
-  if (!s_flag) return;
-  const int r_end = min(o_end * kOctet, p.s.M);
-  for (int r = o_begin * kOctet + threadIdx.x; r < r_end; r += blockDim.x) {
-    float sum = 0.f;
-    for (int t = 0; t < nvs; ++t) sum += __ldcg(p.partial + size_t(t) * Mpad + r);
-    p.y[r] = sum;
-  }
+// y[r] = sum over the nvs partials of row r, in (kernel, slab) order.  A
+// separate grid, so that no CTA of the main kernel waits on another: its
+// dependency wait returns once every partial of the previous grid is written.
+__global__ void __launch_bounds__(256) gemv_combine_kernel(const float* __restrict__ partial, float* __restrict__ y,
+                                                           int M, int Mpad, int nvs) {
+  allow_dependents();
+  grid_dependency_wait();
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= M) return;
+  float sum = 0.f;
+  for (int t = 0; t < nvs; ++t) sum += __ldcg(partial + size_t(t) * Mpad + r);
+  y[r] = sum;
 }
 
 // ---------------------------------------------------------------------------
@@ -411,19 +400,17 @@ inline GemvPlan gemv_plan(const Shape& s, int sm_count, int nk) {
   int cps = sm_count / (pl.nslab * nk);
   if (cps < 1) cps = 1;
   if (cps > s.O) cps = s.O;
-  if (cps > int(kMaxCps)) cps = int(kMaxCps);
   pl.cps = cps;
   return pl;
 }
 
-// Workspace: the first kCounterBytes hold one arrival counter per row range
-// (at most kMaxCps ranges); calls leave them at zero.  Per-CTA partial sums
-// follow.  The counter block has a fixed size so that calls of any shape can
-// share one workspace.
+// Workspace: the per-CTA partial sums [nslab * nk][O * 8] (fp32), written and
+// read by every call; nothing in it survives a call, so it needs no
+// initialisation and any call may reuse it.
 static size_t workspace_bytes_for(const Shape& s, int nk) {
   const size_t nvs = size_t((s.N + kSlabCols - 1) / kSlabCols) * nk;
   if (nvs <= 1) return 0;
-  return kCounterBytes + nvs * size_t(s.O) * kOctet * sizeof(float);
+  return nvs * size_t(s.O) * kOctet * sizeof(float);
 }
 size_t gemv_lut_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, 1); }
 size_t gemv_svid_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, s.K); }
@@ -444,18 +431,30 @@ static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
   cfg.dynamicSmemBytes = G::kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, p);
   if (e != cudaSuccess) return e;
+  const int nvs = p.nslab * (SV ? p.nk : 1);
+  if (nvs > 1) {
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3((p.s.M + 255) / 256);
+    c2.blockDim = dim3(256);
+    c2.stream = stream;
+    c2.attrs = attr;
+    c2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c2, gemv_combine_kernel, static_cast<const float*>(p.partial), p.y, p.s.M,
+                           p.s.O * kOctet, nvs);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
@@ -474,12 +473,7 @@ static GemvParams make_params(const uint8_t* packed, const Shape& s, const void*
   p.cps = pl.cps;
   p.nk = nk;
   p.weights_static = weights_static ? 1 : 0;
-  p.partial = nullptr;
-  p.counter = nullptr;
-  if (pl.nslab * nk > 1) {
-    p.counter = static_cast<unsigned*>(workspace);
-    p.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + kCounterBytes);
-  }
+  p.partial = pl.nslab * nk > 1 ? static_cast<float*>(workspace) : nullptr;
   return p;
 }
 

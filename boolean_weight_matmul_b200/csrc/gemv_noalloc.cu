@@ -1,7 +1,7 @@
 // mbok_gemv_noalloc: the decode GEMV for callers that cannot allocate device
-// memory.  Its scratch (the per-slab partial sums and arrival counters that
-// mbok_gemv keeps in a caller-provided workspace) lives in a fixed-size array
-// compiled into this library instead.  The library allocates nothing here.
+// memory.  Its scratch (the per-slab partial sums that mbok_gemv keeps in a
+// caller-provided workspace) lives in a fixed-size array compiled into this
+// library instead.  The library allocates nothing here.
 #include "mbok_common.cuh"
 
 namespace mbok {
@@ -21,10 +21,6 @@ using namespace mbok;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MBOK_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-
-// The arrival counters occupy the first bytes of any GEMV workspace; they must
-// read zero when a call starts.
-constexpr size_t kCounterBytesToClear = 1024 * sizeof(unsigned);
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
@@ -68,8 +64,6 @@ extern "C" int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, 
   if (need > 0) {
     scratch = scratch_address();
     if (scratch == nullptr) return MBOK_ERR_CUDA;
-    // The array keeps whatever the previous call left: clear the counters.
-    if (cudaMemsetAsync(scratch, 0, kCounterBytesToClear, st) != cudaSuccess) return MBOK_ERR_CUDA;
   }
   if (launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32, batch, y,
                   scratch, st) != cudaSuccess)

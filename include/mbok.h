@@ -82,10 +82,11 @@ size_t mbok_packed_bytes(int K, int M, int N);
 size_t mbok_alpha_elems(int K, int M, int N);
 
 /* Bytes of device workspace mbok_gemv needs for (K, M, N, batch).  The caller
- * allocates it (256-byte aligned), zero-fills it ONCE before its first use,
- * and may reuse it for any later call with the same or smaller requirement
- * on the same stream; calls leave it zero-filled where that matters.  Calls
- * that share one workspace must not run concurrently. */
+ * allocates it (256-byte aligned; no initialisation needed) and may reuse it
+ * for any later call with the same or smaller requirement.  It holds the
+ * per-CTA partial sums of one call, which a second, small launch of the same
+ * call adds up in a fixed order.  Calls that share one workspace must not run
+ * concurrently (calls in one stream are fine). */
 size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch);
 
 /* Pack K sign matrices into layout 1.
@@ -227,16 +228,20 @@ int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t*
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);
 
-/* Promise (on = 1) or withdraw (on = 0, the default) for this process that
- * the packed bits and scales passed to later mbok_gemv / mbok_gemv_noalloc
- * calls are never written by work that may still run on the device when the
- * GEMV is launched -- true for inference with resident weights.  With the
- * promise the lookup kernels copy their first weight tiles into shared
- * memory before waiting for the preceding launch in the stream (launches
- * overlap through programmatic dependent launch), hiding the weights' first
- * DRAM latency behind that launch's tail.  Activations, outputs and the
- * workspace are ordered after the preceding launch either way.  Results do
- * not change.  Returns MBOK_ERR_INVALID_ARG for other values. */
+/* Whether the lookup GEMV kernels may read their weights (packed bits and
+ * scales) before waiting for the preceding launch in the stream.  GEMV
+ * launches use programmatic dependent launch: a GEMV may start while the
+ * kernel before it finishes, if that kernel signalled early
+ * (griddepcontrol.launch_dependents); everything it reads after its wait is
+ * ordered after that kernel.  With on = 1 (the default) the first weight
+ * tiles are copied into shared memory before the wait, hiding their DRAM
+ * latency behind the preceding kernel's tail; activations, outputs and the
+ * workspace are always touched after the wait.  This is safe unless a kernel
+ * that signals early writes the weights right before a GEMV -- no kernel of
+ * this library does (the ones that write weights never signal early, so a
+ * GEMV after them starts only when they are complete).  on = 0 keeps every
+ * read after the wait.  Results do not change.  Process-wide; returns
+ * MBOK_ERR_INVALID_ARG for other values. */
 int mbok_gemv_set_static_weights(int on);
 
 /* mbok_gemv without a workspace argument, for callers that cannot allocate

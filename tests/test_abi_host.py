@@ -52,7 +52,7 @@ def test_sizes(L):
     assert L.mbok_packed_bytes(0, 8, 128) == 0
     assert L.mbok_packed_bytes(1, 8, 100) == 0
     assert L.mbok_gemv_workspace_bytes(3, 4096, 512, 1) == 0       # one slab: no workspace
-    assert L.mbok_gemv_workspace_bytes(3, 4096, 4096, 1) > 8 * 4096 * 4
+    assert L.mbok_gemv_workspace_bytes(3, 4096, 4096, 1) >= 8 * 4096 * 4
     assert L.mbok_gemv_workspace_bytes(3, 4096, 4096, 17) == 0
 
 
@@ -112,8 +112,8 @@ def test_gemv_kernel_choice(L):
 
 def test_gemv_static_weights_switch(L):
     assert L.mbok_gemv_set_static_weights(2) == 1 and L.mbok_gemv_set_static_weights(-1) == 1
-    assert L.mbok_gemv_set_static_weights(1) == 0
     assert L.mbok_gemv_set_static_weights(0) == 0
+    assert L.mbok_gemv_set_static_weights(1) == 0      # the default
 
 
 def test_gemv_svid_argument_errors(L):

@@ -301,6 +301,7 @@ def test_gemv_static_weights_same_bits(M, N):
     x = wl.x_normal(1, N, 103)
     p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
     with mb.gemv_kernel(mb.GEMV_LOOKUP):
+        mb.gemv_set_static_weights(False)
         y0 = gemv_gpu(p, al, K, M, N, x, "bf16")
         mb.gemv_set_static_weights(True)
         try:
@@ -318,7 +319,7 @@ def test_gemv_static_weights_same_bits(M, N):
                     cur = (y * 0.05).to(torch.bfloat16)
             torch.cuda.synchronize()
         finally:
-            mb.gemv_set_static_weights(False)
+            mb.gemv_set_static_weights(True)   # the default
     assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
     assert_close(y1, *O.linear(O.pack_signs(s), a, K, M, N, x, "bf16"), GEMV_REL_L2, "static weights")
     if M == N:
