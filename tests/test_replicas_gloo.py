@@ -1,7 +1,7 @@
-"""The multi-GPU path of the benchmark runs independent replicas (the layer
-does not shard in this build): each rank times its own step and the job
-reports the units of all ranks over the slowest rank's time.  Checked here
-with two gloo ranks on the CPU."""
+"""The multi-GPU path of the benchmark runs independent replicas (one GPU
+holds a layer; no collective is on the data path): each rank times its own
+step and the job reports the units of all ranks over the slowest rank's
+time.  Checked here with two gloo ranks on the CPU."""
 import os
 import socket
 import sys
