@@ -14,7 +14,10 @@
  *
  * Conventions for every call
  *  - All data pointers are DEVICE pointers owned by the caller.  The library
- *    allocates nothing, keeps no state between calls and never synchronises.
+ *    allocates nothing and never synchronises (except
+ *    mbok_read_device_errors); between calls it keeps only cached kernel
+ *    attributes and two process-wide switches (mbok_gemv_set_kernel,
+ *    mbok_gemv_set_static_weights).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued on it; results are ready when the stream reaches them.
  *  - Return value: an mbok_status.  Argument errors are detected on the host
@@ -219,9 +222,9 @@ int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t*
  * devices, all later calls):
  *   MBOK_GEMV_AUTO (default): lookup tables for one vector, tensor cores for
  *     more;
- *   MBOK_GEMV_LOOKUP: lookup tables (8-bit tables over 512-column slabs,
- *     slabs combined across CTAs through the workspace), one launch per
- *     vector;
+ *   MBOK_GEMV_LOOKUP: lookup tables (8-bit tables over 512-column slabs;
+ *     the slabs' partial sums are added by a second small launch through the
+ *     workspace), once per vector;
  *   MBOK_GEMV_TENSOR: tensor cores for any batch.
  * Both kernels meet the accuracy stated for mbok_gemv; results differ in
  * rounding.  Not synchronised with calls in flight on other host threads.
@@ -263,8 +266,8 @@ int mbok_gemv_set_static_weights(int on);
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before any
  *    CUDA stream capture on that device.
- *  - Each call first clears, on `stream`, the part of the array that must
- *    start at zero; the rest keeps what the previous call left.
+ *  - Nothing in the array outlives a call (each call writes its partial sums
+ *    before reading them), so it needs no clearing.
  *  - All calls in the process share the one array: calls that may overlap on
  *    the GPU (different streams without ordering, or several host threads)
  *    race and give wrong results.  Order them on one stream. */
@@ -274,10 +277,11 @@ int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int 
 /* Diagnostic: waits inside the library's kernels are bounded (about a second);
  * a kernel that gives up records a flag and returns early instead of hanging.
  * Writes the flags accumulated on the current device since the last call to
- * *flags (0 = none; bit 0 = a decode-GEMV copy never completed; bit 1 = a
- * prefill-GEMM pipeline wait gave up; bit 2 = a tensor-core GEMV copy wait
- * gave up, in which case that launch stored no outputs) and clears them.  Synchronises the
- * device.  Returns MBOK_ERR_CUDA if the flags cannot be read. */
+ * *flags (0 = none; bit 1 = a prefill-GEMM pipeline wait gave up; bit 2 = a
+ * tensor-core GEMV copy wait gave up, in which case that launch stored no
+ * outputs; bit 0 is reserved and stays 0: the lookup-table GEMV never waits)
+ * and clears them.  Synchronises the device.  Returns MBOK_ERR_CUDA if the
+ * flags cannot be read. */
 int mbok_read_device_errors(unsigned* flags);
 
 /* Self-check of the bounded waits that the pipelined kernels use: launches
