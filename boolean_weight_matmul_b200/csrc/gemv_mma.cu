@@ -413,8 +413,12 @@ __device__ __forceinline__ bool mma_slice(const GemvMmaParams& p, MmaCtx& c, Mma
   return true;
 }
 
-template <int K, int NT, bool XF32>
-__global__ void __launch_bounds__(kMmaThreads, (NT == 2 && K >= 3) ? 1 : 2) gemv_mma_kernel(GemvMmaParams p) {
+// MINB: CTAs per SM the register budget is cut for -- 3 for grids large
+// enough to fill three per SM (more warps to hide latency), else 2 (the
+// scheduler would otherwise crowd a small grid onto fewer SMs); 1 for the
+// register-heavy variants with two 8-column tiles and K >= 3.
+template <int K, int NT, bool XF32, int MINB>
+__global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaParams p) {
   using G = MmaGeom<K, NT, XF32>;
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int stage_bytes = G::kStage;
@@ -549,9 +553,9 @@ __global__ void __launch_bounds__(kMmaThreads, (NT == 2 && K >= 3) ? 1 : 2) gemv
 // Host side
 // ---------------------------------------------------------------------------
 
-template <int K, int NT, bool XF32>
+template <int K, int NT, bool XF32, int MINB>
 static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
-  auto fn = gemv_mma_kernel<K, NT, XF32>;
+  auto fn = gemv_mma_kernel<K, NT, XF32, MINB>;
   using G = MmaGeom<K, NT, XF32>;
   static bool attr_set = false;   // set once, outside any stream capture
   if (!attr_set) {
@@ -577,8 +581,13 @@ static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
 template <int K>
 static cudaError_t launch_mma_nt(const GemvMmaParams& p, bool x_f32, cudaStream_t stream) {
   const int cols = x_f32 ? 3 * p.nb : p.nb;
-  if (cols <= 8) return x_f32 ? launch_mma_k<K, 1, true>(p, stream) : launch_mma_k<K, 1, false>(p, stream);
-  return x_f32 ? launch_mma_k<K, 2, true>(p, stream) : launch_mma_k<K, 2, false>(p, stream);
+  const bool big_grid = (p.s.O + 1) / 2 >= 3 * device_sm_count();
+  if (cols <= 8) {
+    if (big_grid) return x_f32 ? launch_mma_k<K, 1, true, 3>(p, stream) : launch_mma_k<K, 1, false, 3>(p, stream);
+    return x_f32 ? launch_mma_k<K, 1, true, 2>(p, stream) : launch_mma_k<K, 1, false, 2>(p, stream);
+  }
+  constexpr int kMinB2 = K >= 3 ? 1 : 2;
+  return x_f32 ? launch_mma_k<K, 2, true, kMinB2>(p, stream) : launch_mma_k<K, 2, false, kMinB2>(p, stream);
 }
 
 // Self-check of the bounded waits: one warp waits, with the kernels' own wait
