@@ -20,10 +20,11 @@
 //    warp), plus the octet's 4 groups x K scale vectors.  The main loop has
 //    no block-wide barrier.  Launches use programmatic dependent launch:
 //    before waiting on the previous grid the kernel prefetches its first
-//    octets into L2 and (unless turned off, because a kernel that lets this
-//    grid start early might write the weights) starts their shared-memory
-//    copies; the read of x and every write happen after the wait.  A chain of
-//    layers thus overlaps one launch's tail with the next launch's weights.
+//    octets and its slice of x into L2 and (unless turned off, because a
+//    kernel that lets this grid start early might write the weights) starts
+//    the octets' shared-memory copies; the read of x and every write happen
+//    after the wait.  A chain of layers thus overlaps one launch's tail with
+//    the next launch's weights.
 //  * Per (row pair, kernel) a lane does four lookups, one packed fp32x2 add
 //    and one packed fp32x2 FMA with the two rows' fp16 group scales.
 //  * The 32 lanes' partial sums of an octet's 8 rows are combined by a
@@ -302,6 +303,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
       else cp_async_commit();   // keep one group per slot
     }
   }
+  // The slab's activations (and input scales) into L2 as well.  This is safe
+  // even when the previous grid writes x: L2 is the device's point of
+  // coherence, so a line fetched early is updated in place by that write, and
+  // the L1-cached read of x below still comes after the wait.
+  const int col0 = q * kUnit + 8 * (warp >> 3);
+  if (warp == 0 && lane_ok) {
+    prefetch_l2(static_cast<const unsigned char*>(p.x) + size_t(q) * kUnit * (XF32 ? 4 : 2));
+    if (SV) prefetch_l2(p.s_in + size_t(kk) * p.s.N + size_t(q) * kUnit);
+  }
   allow_dependents();
   // x, the workspace and (unless static) the weights may be written by the
   // previous grid: wait for it.
@@ -309,7 +319,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
 
   // x first: its load must not queue behind this warp's weight copies.
   float xv[8];
-  const int col0 = q * kUnit + 8 * (warp >> 3);
   load_x8<XF32>(p.x, col0, lane_ok, xv);
   if (SV && lane_ok) {
     // rank-1 form: the kernel's input scale, applied before the tables
