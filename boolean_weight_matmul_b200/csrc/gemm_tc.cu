@@ -31,9 +31,7 @@
 // elements of one output row of Y.
 // Every mbarrier wait is bounded (1 s); on timeout the CTA records an error
 // flag, drains what it issued (bounded), frees its tensor memory and exits.
-#include <cuda.h>
-
-#include "mbok_common.cuh"
+#include "tc_common.cuh"
 
 namespace mbok {
 
@@ -54,13 +52,9 @@ constexpr int kTcEpiWarp0 = 2 + kTcUnpackWarps;                 // 4 epilogue wa
 constexpr int kTcThreads = (2 + kTcUnpackWarps + 4) * 32;       // TMA, MMA, 16 unpack, 4 epilogue
 constexpr int kTcSmem = kTcStages * kTcStageBytes + 1024 + 256;  // + alignment + barriers
 constexpr unsigned kTcTmemCols = 512;      // row halves 0 and 1: columns 0.. and 256..
-constexpr unsigned long long kTcWaitNs = 1000000000ull;
-constexpr unsigned long long kTcDrainNs = 200000000ull;
 
 // Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=n.
-inline uint32_t tc_idesc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kTcHalf >> 4) << 24);
-}
+inline uint32_t tc_idesc(int n) { return tc_idesc_bf16(kTcHalf, n); }
 
 __device__ unsigned int g_gemm_error;
 
@@ -73,90 +67,6 @@ struct TcParams {
   int n_tile;       // tokens per CTA tile (multiple of 16, <= kTcTokens)
   uint32_t idesc;   // instruction descriptor for N = n_tile
 };
-
-// ---------------------------------------------------------------------------
-// PTX helpers
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t tc_smem(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long tc_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;\n" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void tc_mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc_smem(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void tc_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tc_smem(bar)) : "memory");
-}
-
-__device__ __forceinline__ void tc_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tc_smem(bar)), "r"(bytes)
-               : "memory");
-}
-
-// Bounded wait for phase `parity`; false on timeout.
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, unsigned parity, unsigned long long limit = kTcWaitNs) {
-  const uint32_t a = tc_smem(bar);
-  unsigned long long t0 = 0;
-  for (unsigned it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((it & 255u) == 0) {
-      const unsigned long long t = tc_ns();
-      if (t0 == 0) t0 = t;
-      else if (t - t0 > limit) return false;
-    }
-  }
-}
-
-__device__ __forceinline__ void tc_tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          tc_smem(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(tc_smem(bar))
-      : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (version 1 for sm_100).
-__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFF);        // start address
-  d |= uint64_t(1) << 16;                      // leading byte offset (unused for swizzled K-major)
-  d |= uint64_t(1024 >> 4) << 32;              // stride byte offset
-  d |= uint64_t(1) << 46;                      // descriptor version
-  d |= uint64_t(2) << 61;                      // SWIZZLE_128B
-  return d;
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  const uint32_t z = 0;
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(tc_smem(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Unpack: 2 rows x 16 columns of W (all K kernels) -> bf16 in the swizzled tile
@@ -408,11 +318,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 // Host side
 // ---------------------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
+EncodeTiledFn tensor_map_encoder() {
   static EncodeTiledFn fn = nullptr;
   if (fn == nullptr) {
     void* ptr = nullptr;
@@ -470,7 +376,7 @@ int tc_token_tile(int M, int T, int sms) {
 // Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
 cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const uint16_t* X,
                            int T, uint16_t* Y, cudaStream_t stream) {
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   const int n_tile = tc_token_tile(s.M, T, device_sm_count());
   const cuuint32_t ones[2] = {1, 1};
