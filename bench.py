@@ -453,7 +453,7 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
     # weight copies per graph that they exceed L2 (>= 150 MB).
     shapes = (("q_proj", 3, 4096, 4096), ("gate", 3, 11008, 4096), ("down", 2, 4096, 11008))
     kernels = (("lookup", mb.GEMV_LOOKUP, True), ("lookup_weights_after_wait", mb.GEMV_LOOKUP, False),
-               ("tensor", mb.GEMV_TENSOR, True), ("tcgen05", mb.GEMV_TCGEN05, True))
+               ("tensor", mb.GEMV_TENSOR, True))
     for (name, K, M, N) in shapes:
         bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
         L = max(8, -(-150_000_000 // bpl))

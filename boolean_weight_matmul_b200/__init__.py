@@ -25,7 +25,6 @@ MAX_BATCH = 16
 GEMV_AUTO = 0
 GEMV_LOOKUP = 1
 GEMV_TENSOR = 2
-GEMV_TCGEN05 = 3
 
 _lib = None
 
@@ -206,7 +205,7 @@ def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=Non
 
 def gemv_set_kernel(kernel: int) -> None:
     """Process-wide kernel choice of gemv / gemv_noalloc (GEMV_AUTO,
-    GEMV_LOOKUP, GEMV_TENSOR or GEMV_TCGEN05)."""
+    GEMV_LOOKUP or GEMV_TENSOR)."""
     _check(lib().mbok_gemv_set_kernel(kernel), "mbok_gemv_set_kernel")
 
 

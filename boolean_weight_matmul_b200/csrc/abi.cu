@@ -25,11 +25,6 @@ cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const
                             float*, cudaStream_t);
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
                         void*, cudaStream_t);
-cudaError_t launch_gemv_tc(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*, void*,
-                           cudaStream_t);
-size_t gemv_tc_workspace_bytes(const Shape&, int);
-unsigned gemv_tc_error_flags();
-size_t gemv_workspace_need(const Shape&, int);
 
 cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
                            uint16_t*, cudaStream_t);
@@ -41,20 +36,10 @@ int gemv_kernel_choice = MBOK_GEMV_AUTO;
 // (see mbok_gemv_set_static_weights).
 bool gemv_weights_static = true;
 
-// Workspace of one GEMV call, whichever kernel the process-wide choice picks:
-// the lookup kernel's slab partials or the tcgen05 kernel's tile partials
-// and split activations.
-size_t gemv_workspace_need(const Shape& s, int batch) {
-  const size_t a = gemv_lut_workspace_bytes(s), b = gemv_tc_workspace_bytes(s, batch);
-  return a > b ? a : b;
-}
-
-// One decode GEMV call: the lookup-table kernel once per vector, or a
+// One decode GEMV call: the lookup-table kernel once per vector, or the
 // tensor-core kernel over the whole batch.
 cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
                         bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
-  if (gemv_kernel_choice == MBOK_GEMV_TCGEN05)
-    return launch_gemv_tc(packed, alpha, s, x, x_f32, batch, y, workspace, stream);
   bool tensor = batch > 1;
   if (gemv_kernel_choice == MBOK_GEMV_LOOKUP) tensor = false;
   if (gemv_kernel_choice == MBOK_GEMV_TENSOR) tensor = true;
@@ -123,7 +108,7 @@ size_t mbok_alpha_elems(int K, int M, int N) {
 
 size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch) {
   if (check_shape(K, M, N) != MBOK_OK || batch < 1 || batch > MBOK_MAX_BATCH) return 0;
-  return gemv_workspace_need(make_shape(K, M, N), batch);
+  return gemv_lut_workspace_bytes(make_shape(K, M, N));
 }
 
 int mbok_pack_bits(const int8_t* signs, int K, int M, int N, uint32_t* packed, void* stream) {
@@ -207,7 +192,7 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
   if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(x, 16) || !aligned(y, 4))
     return MBOK_ERR_ALIGN;
   const Shape s = make_shape(K, M, N);
-  const size_t need = gemv_workspace_need(s, batch);
+  const size_t need = gemv_lut_workspace_bytes(s);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
     return MBOK_ERR_WORKSPACE;
   return from_cuda(launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32,
@@ -221,7 +206,7 @@ int mbok_gemv_set_static_weights(int on) {
 }
 
 int mbok_gemv_set_kernel(int kernel) {
-  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TCGEN05) return MBOK_ERR_INVALID_ARG;
+  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TENSOR) return MBOK_ERR_INVALID_ARG;
   gemv_kernel_choice = kernel;
   return MBOK_OK;
 }
@@ -268,9 +253,8 @@ int mbok_read_device_errors(unsigned* flags) {
   const unsigned g = gemv_error_flags();
   const unsigned m = gemm_error_flags();
   const unsigned t = gemv_mma_error_flags();
-  const unsigned c = gemv_tc_error_flags();
-  if (g == ~0u || m == ~0u || t == ~0u || c == ~0u) return MBOK_ERR_CUDA;
-  *flags = (g ? 1u : 0u) | (m ? 2u : 0u) | ((t | c) ? 4u : 0u);
+  if (g == ~0u || m == ~0u || t == ~0u) return MBOK_ERR_CUDA;
+  *flags = (g ? 1u : 0u) | (m ? 2u : 0u) | (t ? 4u : 0u);
   return MBOK_OK;
 }
 

@@ -9,7 +9,7 @@ cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const voi
                         void*, cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t, bool);
-size_t gemv_workspace_need(const Shape&, int);
+size_t gemv_lut_workspace_bytes(const Shape&);
 }  // namespace mbok
 
 using namespace mbok;
@@ -56,7 +56,7 @@ extern "C" int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, 
       (reinterpret_cast<uintptr_t>(x) & a16) || (reinterpret_cast<uintptr_t>(y) & 3))
     return MBOK_ERR_ALIGN;
   const Shape s = make_shape(K, M, N);
-  const size_t need = gemv_workspace_need(s, batch);
+  const size_t need = gemv_lut_workspace_bytes(s);
   if (need > size_t(MBOK_NOALLOC_SCRATCH_BYTES)) return MBOK_ERR_SCRATCH_LIMIT;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);

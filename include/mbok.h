@@ -69,7 +69,6 @@ typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
 #define MBOK_GEMV_AUTO 0
 #define MBOK_GEMV_LOOKUP 1
 #define MBOK_GEMV_TENSOR 2
-#define MBOK_GEMV_TCGEN05 3
 /* Size of the scratch array built into the library for mbok_gemv_noalloc. */
 #define MBOK_NOALLOC_SCRATCH_BYTES (4u << 20)
 
@@ -85,13 +84,11 @@ size_t mbok_packed_bytes(int K, int M, int N);
 /* fp16 elements of the blocked scales: ceil(M/8)*8*(N/128)*K.  0 on bad shape. */
 size_t mbok_alpha_elems(int K, int M, int N);
 
-/* Bytes of device workspace mbok_gemv needs for (K, M, N, batch), whichever
- * kernel mbok_gemv_set_kernel selects.  The caller allocates it (256-byte
- * aligned; no initialisation needed) and may reuse it for any later call
- * with the same or smaller requirement.  It holds the per-CTA partial sums
- * of one call, which a second, small launch of the same call adds up in a
- * fixed order (and, for fp32 activations on the tcgen05 kernel, their bf16
- * parts).  Calls that share one workspace must not run
+/* Bytes of device workspace mbok_gemv needs for (K, M, N, batch).  The caller
+ * allocates it (256-byte aligned; no initialisation needed) and may reuse it
+ * for any later call with the same or smaller requirement.  It holds the
+ * per-CTA partial sums of one call, which a second, small launch of the same
+ * call adds up in a fixed order.  Calls that share one workspace must not run
  * concurrently (calls in one stream are fine). */
 size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch);
 
@@ -228,14 +225,8 @@ int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t*
  *   MBOK_GEMV_LOOKUP: lookup tables (8-bit tables over 512-column slabs;
  *     the slabs' partial sums are added by a second small launch through the
  *     workspace), once per vector;
- *   MBOK_GEMV_TENSOR: tensor cores (mma.sync, 16-row tiles) for any batch;
- *   MBOK_GEMV_TCGEN05: tensor cores through tcgen05 for any batch: the sign
- *     tiles are written into tensor memory and multiplied there, 128-row
- *     tiles shared out over the SMs in equal runs of (tile, group) units; the
- *     partial row sums are added by a second small launch through the
- *     workspace (fp32 input: a first small launch splits x into its three
- *     exact bf16 parts, also in the workspace).
- * All kernels meet the accuracy stated for mbok_gemv; results differ in
+ *   MBOK_GEMV_TENSOR: tensor cores for any batch.
+ * Both kernels meet the accuracy stated for mbok_gemv; results differ in
  * rounding.  Not synchronised with calls in flight on other host threads.
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);

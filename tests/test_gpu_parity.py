@@ -218,10 +218,10 @@ def test_gemv_deterministic():
 # The two GEMV kernels, each forced for every batch size
 # --------------------------------------------------------------------------
 
-KERNELS = {"lookup": 1, "tensor": 2, "tcgen05": 3}
+KERNELS = {"lookup": 1, "tensor": 2}
 
 
-@pytest.mark.parametrize("kernel", ["lookup", "tensor", "tcgen05"])
+@pytest.mark.parametrize("kernel", ["lookup", "tensor"])
 @pytest.mark.parametrize("K", [1, 2, 3, 4])
 @pytest.mark.parametrize("M,N,batch", [(1, 128, 1), (7, 256, 3), (13, 640, 5), (129, 1024, 2),
                                        (64, 1536, 16), (24, 384, 6)])
@@ -233,19 +233,17 @@ def test_gemv_kernel_small_shapes(kernel, K, M, N, batch):
             assert_close(y, y_ref, E, GEMV_REL_L2, f"{kernel} K={K} M={M} N={N} b={batch} {x_dtype}")
 
 
-@pytest.mark.parametrize("kernel", ["tensor", "tcgen05"])
 @pytest.mark.parametrize("batch", [1, 5, 6, 11, 16])
-def test_gemv_tensor_f32_batches(kernel, batch):
-    # fp32 activations take three bf16 columns (rows of B) each.
+def test_gemv_tensor_f32_batches(batch):
+    # fp32 activations take three bf16 columns each: 5 vectors per launch.
     import boolean_weight_matmul_b200 as mb
-    with mb.gemv_kernel(KERNELS[kernel]):
-        y, y_ref, E = _gemv_case(3, 300, 768, batch, "f32", 6500 + batch, "decaying")
-    assert_close(y, y_ref, E, GEMV_REL_L2, f"{kernel} f32 batch={batch}")
+    with mb.gemv_kernel(mb.GEMV_TENSOR):
+        y, y_ref, E = _gemv_case(3, 40, 768, batch, "f32", 6500 + batch, "decaying")
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"tensor f32 batch={batch}")
 
 
-@pytest.mark.parametrize("kernel", ["tensor", "tcgen05"])
 @pytest.mark.parametrize("batch", [1, 16])
-def test_gemv_tensor_q_proj_full(kernel, batch):
+def test_gemv_tensor_q_proj_full(batch):
     # LLaMA-7B q_proj K=3 on the tensor-core kernel, every output row checked.
     import torch
     import boolean_weight_matmul_b200 as mb
@@ -255,27 +253,24 @@ def test_gemv_tensor_q_proj_full(kernel, batch):
     a = wl.alpha_decaying(K, M, N, wl.seed_of(2, 0, 1))
     x = wl.x_normal(batch, N, wl.seed_of(2, 0, 2))
     packed = to_dev(words.view(np.int32))
-    with mb.gemv_kernel(KERNELS[kernel]):
+    with mb.gemv_kernel(mb.GEMV_TENSOR):
         y = gemv_gpu(packed, alpha_blocked_gpu(a, K, M, N), K, M, N, x, "bf16")
     y_ref, E = O.linear(words, a, K, M, N, x, "bf16")
-    assert_close(y, y_ref, E, GEMV_REL_L2, f"{w.name} {kernel} b{batch}")
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"{w.name} tensor b{batch}")
     del packed
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("kernel", ["tensor", "tcgen05"])
 @pytest.mark.parametrize("name,M,N,batch", [("gate", 11008, 4096, 4), ("down", 4096, 11008, 16),
                                             ("gate13b", 13824, 5120, 16)])
-def test_gemv_tensor_mlp_sampled(kernel, name, M, N, batch):
-    import boolean_weight_matmul_b200 as mb
+def test_gemv_tensor_mlp_sampled(name, M, N, batch):
     K = 3 if name == "gate" else (2 if name == "down" else 4)
     rows = np.sort(np.random.default_rng(M + batch).choice(M, 256, replace=False))
-    with mb.gemv_kernel(KERNELS[kernel]):
-        y, y_ref, E = _gemv_case(K, M, N, batch, "bf16", 7000 + M + N, "decaying", rows=rows)
-    assert_close(y, y_ref, E, GEMV_REL_L2, f"{kernel} {name} b{batch}")
+    y, y_ref, E = _gemv_case(K, M, N, batch, "bf16", 7000 + M + N, "decaying", rows=rows)
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"tensor {name} b{batch}")
 
 
-@pytest.mark.parametrize("kernel", ["lookup", "tensor", "tcgen05"])
+@pytest.mark.parametrize("kernel", ["lookup", "tensor"])
 def test_gemv_kernel_flip_invariance_bitwise(kernel):
     # Negated signs (exact) times negated scales: the same y bit for bit.
     import boolean_weight_matmul_b200 as mb
@@ -356,27 +351,6 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
     assert np.array_equal(y0[:9].view(np.uint32), y9.view(np.uint32))
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
-
-
-def test_gemv_tcgen05_deterministic_and_batch_independent():
-    # tcgen05 kernel: every bf16 batch uses the same MMA shape (N = 16 rows of
-    # B) and the same split of (tile, group) units over the CTAs, so a vector's
-    # result is the same bits whatever its batch neighbours, and run to run.
-    import boolean_weight_matmul_b200 as mb
-    K, M, N = 3, 1000, 4096
-    s = wl.random_signs(K, M, N, 94)
-    a = wl.alpha_decaying(K, M, N, 95)
-    x = wl.x_normal(16, N, 96)
-    p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
-    with mb.gemv_kernel(mb.GEMV_TCGEN05):
-        y0 = gemv_gpu(p, al, K, M, N, x, "bf16")
-        y1 = gemv_gpu(p, al, K, M, N, x, "bf16")
-        y9 = gemv_gpu(p, al, K, M, N, x[:9], "bf16")
-        y_one = gemv_gpu(p, al, K, M, N, x[5:6], "bf16")
-    assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
-    assert np.array_equal(y0[:9].view(np.uint32), y9.view(np.uint32))
-    assert np.array_equal(y0[5].view(np.uint32), y_one[0].view(np.uint32))
-    assert_close(y0, *O.linear(O.pack_signs(s), a, K, M, N, x, "bf16"), GEMV_REL_L2, "tcgen05 b16")
 
 
 def test_gemv_fused_projections_equal_separate_calls():
