@@ -83,16 +83,28 @@ def _check(status: int, what: str) -> None:
         raise MbokError(what, status)
 
 
-def _ptr(t) -> int | None:
-    if t is None:
-        return None
-    if isinstance(t, int):
-        return t
-    if not t.is_cuda:
-        raise ValueError("MBOK operates on CUDA tensors only")
-    if not t.is_contiguous():
-        raise ValueError("MBOK needs contiguous tensors")
-    return t.data_ptr()
+def _ptrs(*ts) -> list:
+    """Device pointers of the arguments (None stays None, an int is taken as a
+    raw device pointer).  Every tensor must be a contiguous CUDA tensor on the
+    current device: the library launches there, and a pointer into another
+    GPU's memory would be dereferenced by its kernels."""
+    dev = None
+    out = []
+    for t in ts:
+        if t is None or isinstance(t, int):
+            out.append(t)
+            continue
+        if not t.is_cuda:
+            raise ValueError("MBOK operates on CUDA tensors only")
+        if not t.is_contiguous():
+            raise ValueError("MBOK needs contiguous tensors")
+        if dev is None:
+            dev = torch.cuda.current_device()
+        if t.device.index != dev:
+            raise ValueError(f"tensor on {t.device} but the current device is cuda:{dev}; "
+                             "MBOK launches on the current device")
+        out.append(t.data_ptr())
+    return out
 
 
 def _stream(stream) -> int | None:
@@ -145,39 +157,42 @@ def zeros_workspace(K: int, M: int, N: int, batch: int = 1, device="cuda") -> to
 # ---- the calls ------------------------------------------------------------
 
 def pack_bits(signs, K, M, N, packed, stream=None) -> None:
-    _check(lib().mbok_pack_bits(_ptr(signs), K, M, N, _ptr(packed), _stream(stream)), "mbok_pack_bits")
+    ps, pp = _ptrs(signs, packed)
+    _check(lib().mbok_pack_bits(ps, K, M, N, pp, _stream(stream)), "mbok_pack_bits")
 
 
 def pack_alpha(alpha_mgk, K, M, N, alpha_out, stream=None) -> None:
-    _check(lib().mbok_pack_alpha(_ptr(alpha_mgk), K, M, N, _ptr(alpha_out), _stream(stream)),
-           "mbok_pack_alpha")
+    pa, po = _ptrs(alpha_mgk, alpha_out)
+    _check(lib().mbok_pack_alpha(pa, K, M, N, po, _stream(stream)), "mbok_pack_alpha")
 
 
 def residual_binarize(W, M, N, K, group, packed, alpha, residual=None, stream=None) -> None:
-    _check(lib().mbok_residual_binarize(_ptr(W), M, N, K, group, _ptr(packed), _ptr(alpha),
-                                        _ptr(residual), _stream(stream)), "mbok_residual_binarize")
+    pw, pp, pa, pr = _ptrs(W, packed, alpha, residual)
+    _check(lib().mbok_residual_binarize(pw, M, N, K, group, pp, pa, pr, _stream(stream)), "mbok_residual_binarize")
 
 
 def svid_binarize(W, M, N, K, iters, packed, s_in, s_out, residual, workspace=None, stream=None) -> None:
     """Successive SVID (see include/mbok.h); allocates its workspace if none is given."""
     if workspace is None:
         workspace = torch.empty(int(lib().mbok_svid_workspace_bytes(M, N)), dtype=torch.uint8, device=W.device)
-    _check(lib().mbok_svid_binarize(_ptr(W), M, N, K, iters, _ptr(packed), _ptr(s_in), _ptr(s_out), _ptr(residual),
-                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+    pw, pp, pi, po, pr, pws = _ptrs(W, packed, s_in, s_out, residual, workspace)
+    _check(lib().mbok_svid_binarize(pw, M, N, K, iters, pp, pi, po, pr, pws,
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "mbok_svid_binarize")
 
 
 def refit_alpha(W, packed, K, M, N, group, alpha_out, stream=None) -> None:
     """Least-squares scales for fixed kernels (see include/mbok.h)."""
-    _check(lib().mbok_refit_alpha(_ptr(W), _ptr(packed), K, M, N, group, _ptr(alpha_out), _stream(stream)),
-           "mbok_refit_alpha")
+    pw, pp, po = _ptrs(W, packed, alpha_out)
+    _check(lib().mbok_refit_alpha(pw, pp, K, M, N, group, po, _stream(stream)), "mbok_refit_alpha")
 
 
 def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=None) -> None:
     ws_bytes = 0 if workspace is None else (workspace.numel() * workspace.element_size()
                                             if isinstance(workspace, torch.Tensor) else 0)
-    _check(lib().mbok_gemv(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype, batch,
-                           _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv")
+    pp, pa, px, py, pws = _ptrs(packed, alpha, x, y, workspace)
+    _check(lib().mbok_gemv(pp, pa, K, M, N, group, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
+           "mbok_gemv")
 
 
 def gemv_svid_workspace_bytes(K: int, M: int, N: int, batch: int = 1) -> int:
@@ -192,15 +207,17 @@ def zeros_svid_workspace(K: int, M: int, N: int, batch: int = 1, device="cuda") 
 def gemv_svid(packed, s_in, s_out, K, M, N, x, x_dtype, batch, y, workspace, stream=None) -> None:
     """Rank-1-scaled layer: y = sum_k s_out[k] * (B_k (s_in[k] * x)) (see include/mbok.h)."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().mbok_gemv_svid(_ptr(packed), _ptr(s_in), _ptr(s_out), K, M, N, _ptr(x), x_dtype, batch,
-                                _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mbok_gemv_svid")
+    pp, pi, po, px, py, pws = _ptrs(packed, s_in, s_out, x, y, workspace)
+    _check(lib().mbok_gemv_svid(pp, pi, po, K, M, N, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
+           "mbok_gemv_svid")
 
 
 def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=None) -> None:
     """mbok_gemv for callers that cannot allocate: scratch comes from the
     library's built-in array (see include/mbok.h)."""
-    _check(lib().mbok_gemv_noalloc(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(x), x_dtype,
-                                   batch, _ptr(y), _stream(stream)), "mbok_gemv_noalloc")
+    pp, pa, px, py = _ptrs(packed, alpha, x, y)
+    _check(lib().mbok_gemv_noalloc(pp, pa, K, M, N, group, px, x_dtype, batch, py, _stream(stream)),
+           "mbok_gemv_noalloc")
 
 
 def gemv_set_kernel(kernel: int) -> None:
@@ -232,8 +249,8 @@ class gemv_kernel:
 
 
 def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:
-    _check(lib().mbok_gemm(_ptr(packed), _ptr(alpha), K, M, N, group, _ptr(X), T, _ptr(Y),
-                           _stream(stream)), "mbok_gemm")
+    pp, pa, px, py = _ptrs(packed, alpha, X, Y)
+    _check(lib().mbok_gemm(pp, pa, K, M, N, group, px, T, py, _stream(stream)), "mbok_gemm")
 
 
 def read_device_errors() -> int:

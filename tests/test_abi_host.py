@@ -152,3 +152,37 @@ def test_svid_binarize_argument_errors(L):
 def test_wait_timeout_check_argument_errors(L):
     assert L.mbok_check_wait_timeout(0, None) == 1
     assert L.mbok_check_wait_timeout(2000000, None) == 1
+
+
+def test_pointer_marshalling_checks_device(monkeypatch):
+    # The binding passes raw device pointers to kernels launched on the
+    # current device, so it refuses CPU, non-contiguous and other-device
+    # tensors before anything reaches the library.  Stand-in tensors keep this
+    # a host-only test.
+    import types
+    import torch
+    import boolean_weight_matmul_b200 as mb
+
+    class Fake:
+        def __init__(self, dev, contiguous=True, cuda=True, ptr=0x1000):
+            self.is_cuda = cuda
+            self.device = types.SimpleNamespace(index=dev, type="cuda" if cuda else "cpu")
+            self._c = contiguous
+            self._p = ptr
+
+        def is_contiguous(self):
+            return self._c
+
+        def data_ptr(self):
+            return self._p
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    assert mb._ptrs(Fake(1, ptr=16), None, 7) == [16, None, 7]
+    with pytest.raises(ValueError, match="current device"):
+        mb._ptrs(Fake(1), Fake(0))
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        mb._ptrs(Fake(None, cuda=False))
+    with pytest.raises(ValueError, match="contiguous"):
+        mb._ptrs(Fake(1, contiguous=False))
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        mb.gemv(torch.zeros(4, dtype=torch.int32), None, 1, 8, 128, 128, None, mb.BF16, 1, None, None)
