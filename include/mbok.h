@@ -13,7 +13,9 @@
  * K Boolean matrix-vector products (same section).
  *
  * Conventions for every call
- *  - All data pointers are DEVICE pointers owned by the caller.  The library
+ *  - All data pointers are DEVICE pointers owned by the caller, in memory of
+ *    the current device (cudaSetDevice): kernels launch there and the library
+ *    does not check where a pointer lives.  The library
  *    allocates nothing and never synchronises (except
  *    mbok_read_device_errors); between calls it keeps only cached kernel
  *    attributes and two process-wide switches (mbok_gemv_set_kernel,
