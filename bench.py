@@ -372,7 +372,9 @@ def run_gpu(a):
 
     del graph
     extras = None
-    if not a.no_extras:
+    # The secondary rows are single-GPU rows: reported at N = 1 only, so a
+    # replica run holds its GPUs just for the headline and end-to-end steps.
+    if not a.no_extras and world == 1:
         del packed, alphas, xs, ys
         torch.cuda.empty_cache()
         extras = run_extras(torch, mb, wl, dev, peaks, a)
