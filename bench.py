@@ -580,6 +580,42 @@ def run_sweep_row(torch, mb, wl, dev, peaks, stream, g, out):
     del mats
     torch.cuda.empty_cache()
 
+    # Each matrix with its own number of kernels (an illustrative allocation,
+    # 3.14 kernels on average: q 3, k 2, v 4, o 3, gate 3, up 3, down 4), and
+    # q/k/v and gate/up each one mbok_gemv_multi launch: 4 launches per layer.
+    alloc = {"q": 3, "k": 2, "v": 4, "o": 3, "gate": 3, "up": 3, "down": 4}
+    groups = (((("q", 5120), ("k", 5120), ("v", 5120)), 5120), ((("o", 5120),), 5120),
+              ((("gate", 13824), ("up", 13824)), 5120), ((("down", 5120),), 13824))
+    calls = []
+    mixed_bytes = 0
+    for _ in range(layers):
+        for (grp, N) in groups:
+            Ks = [alloc[n] for (n, _) in grp]
+            Ms = [M for (_, M) in grp]
+            ps, als = [], []
+            for (K_, M_) in zip(Ks, Ms):
+                ps.append(torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K_, M_, N) // 4,), dtype=torch.int32,
+                                        device=dev, generator=g))
+                al = torch.empty(mb.alpha_elems(K_, M_, N), dtype=torch.float16, device=dev)
+                al.copy_((torch.rand(al.shape, device=dev, generator=g) + 0.5) * 0.01)
+                als.append(al)
+                mixed_bytes += mb.packed_bytes(K_, M_, N) + 2 * mb.alpha_elems(K_, M_, N)
+            calls.append((ps, als, Ks, Ms, N))
+    ws_m = torch.zeros(max(max(mb.gemv_multi_workspace_bytes(c[2], c[3], c[4]) for c in calls), 256),
+                       dtype=torch.uint8, device=dev)
+    ymix = {sum(c[3]): torch.empty(1, sum(c[3]), dtype=torch.float32, device=dev) for c in calls}
+
+    def sweep_mixed():
+        for (ps, als, Ks, Ms, N) in calls:
+            mb.gemv_multi(ps, als, Ks, Ms, N, 128, xin[N], mb.BF16, 1, ymix[sum(Ms)], ws_m, stream=stream)
+    ms, gr = time_graph(torch, sweep_mixed, 5, 2, stream)
+    gbs = mixed_bytes / (ms * 1e-3) / 1e9
+    out["sweep_llama13b_mixedk_40x4_multi_b1"] = {
+        "ms_per_token": ms, "tokens_per_s": 1e3 / ms, "bytes_per_token": mixed_bytes, "gbs": gbs,
+        "frac_of_hbm": gbs / peaks["hbm_gbs"], "launches": len(calls), "kernels": alloc}
+    del gr, calls
+    torch.cuda.empty_cache()
+
 
 def run_conversion_rows(torch, mb, wl, dev, peaks, stream, g, out, rows):
     # Residual binarisation, LLaMA-7B gate 11008 x 4096, K=3.

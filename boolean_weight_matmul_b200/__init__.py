@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
             "mbok_refit_alpha": ([vp, vp, i, i, i, i, vp, vp], i),
             "mbok_svid_workspace_bytes": ([i, i], sz),
             "mbok_svid_binarize": ([vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp], i),
+            "mbok_gemv_multi_workspace_bytes": ([i, vp, vp, i], sz),
+            "mbok_gemv_multi": ([i, vp, vp, vp, vp, i, i, vp, i, i, vp, vp, sz, vp], i),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -193,6 +195,41 @@ def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=
     pp, pa, px, py, pws = _ptrs(packed, alpha, x, y, workspace)
     _check(lib().mbok_gemv(pp, pa, K, M, N, group, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
            "mbok_gemv")
+
+
+def _int_array(vals):
+    arr = (ctypes.c_int * len(vals))(*[int(v) for v in vals])
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+def gemv_multi_workspace_bytes(K_list, M_list, N: int) -> int:
+    ka, kp = _int_array(K_list)
+    ma, mp = _int_array(M_list)
+    return int(lib().mbok_gemv_multi_workspace_bytes(len(K_list), kp, mp, N))
+
+
+def zeros_multi_workspace(K_list, M_list, N: int, device="cuda") -> torch.Tensor:
+    n = max(gemv_multi_workspace_bytes(K_list, M_list, N), 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gemv_multi(packed_list, alpha_list, K_list, M_list, N, group, x, x_dtype, batch, y, workspace,
+               stream=None) -> None:
+    """Several matrices sharing x, each with its own K and M, in one launch per
+    vector; y holds their outputs one after another (see include/mbok.h)."""
+    n = len(packed_list)
+    if not (len(alpha_list) == len(K_list) == len(M_list) == n):
+        raise ValueError("gemv_multi: one packed, alpha, K and M per matrix")
+    ptrs = _ptrs(*packed_list, *alpha_list, x, y, workspace)
+    pp = (ctypes.c_void_p * n)(*ptrs[:n])
+    pa = (ctypes.c_void_p * n)(*ptrs[n:2 * n])
+    px, py, pws = ptrs[2 * n:]
+    ka, kp = _int_array(K_list)
+    ma, mp = _int_array(M_list)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mbok_gemv_multi(n, ctypes.cast(pp, ctypes.c_void_p), ctypes.cast(pa, ctypes.c_void_p), kp, mp,
+                                 N, group, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
+           "mbok_gemv_multi")
 
 
 def gemv_svid_workspace_bytes(K: int, M: int, N: int, batch: int = 1) -> int:

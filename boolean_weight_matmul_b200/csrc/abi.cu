@@ -26,6 +26,10 @@ cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
                         void*, cudaStream_t);
 
+cudaError_t launch_gemv_lut_multi(int, const uint8_t* const*, const uint16_t* const*, const int*, const int*, int,
+                                  const void*, bool, float*, void*, cudaStream_t, bool);
+size_t gemv_multi_workspace_bytes(int, const int*, const int*, int);
+
 cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
                            uint16_t*, cudaStream_t);
 unsigned gemm_error_flags();
@@ -197,6 +201,58 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
     return MBOK_ERR_WORKSPACE;
   return from_cuda(launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32,
                                batch, y, workspace, as_stream(stream)));
+}
+
+// Argument checks of the multi-matrix GEMV's shape arrays; MBOK_OK or the
+// first failing status, and the total row count in *rows.
+static int check_multi(int nseg, const int* K, const int* M, int N, long long* rows) {
+  if (nseg < 1 || nseg > 8 || K == nullptr || M == nullptr) return MBOK_ERR_INVALID_ARG;
+  long long total = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int st = check_shape(K[i], M[i], N);
+    if (st != MBOK_OK) return st;
+    total += M[i];
+  }
+  if (total > (1 << 22)) return MBOK_ERR_SHAPE;
+  *rows = total;
+  return MBOK_OK;
+}
+
+size_t mbok_gemv_multi_workspace_bytes(int nseg, const int* K, const int* M, int N) {
+  long long rows = 0;
+  if (check_multi(nseg, K, M, N, &rows) != MBOK_OK) return 0;
+  return gemv_multi_workspace_bytes(nseg, K, M, N);
+}
+
+int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* const* alpha, const int* K,
+                    const int* M, int N, int group, const void* x, int x_dtype, int batch, float* y,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  long long rows = 0;
+  const int st = check_multi(nseg, K, M, N, &rows);
+  if (st != MBOK_OK) return st;
+  if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
+  if (packed == nullptr || alpha == nullptr || x == nullptr || y == nullptr) return MBOK_ERR_INVALID_ARG;
+  if (x_dtype != MBOK_F32 && x_dtype != MBOK_BF16) return MBOK_ERR_INVALID_ARG;
+  if (batch < 1 || batch > MBOK_MAX_BATCH) return MBOK_ERR_INVALID_ARG;
+  for (int i = 0; i < nseg; ++i) {
+    if (packed[i] == nullptr || alpha[i] == nullptr) return MBOK_ERR_INVALID_ARG;
+    if (!aligned(packed[i], 16) || !aligned(alpha[i], 16)) return MBOK_ERR_ALIGN;
+  }
+  if (!aligned(x, 16) || !aligned(y, 4)) return MBOK_ERR_ALIGN;
+  const size_t need = gemv_multi_workspace_bytes(nseg, K, M, N);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
+    return MBOK_ERR_WORKSPACE;
+  const uint8_t* p8[8];
+  for (int i = 0; i < nseg; ++i) p8[i] = reinterpret_cast<const uint8_t*>(packed[i]);
+  const size_t xbytes = (x_dtype == MBOK_F32) ? 4 : 2;
+  for (int b = 0; b < batch; ++b) {
+    const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
+    const cudaError_t e = launch_gemv_lut_multi(nseg, p8, alpha, K, M, N, xb, x_dtype == MBOK_F32,
+                                                y + size_t(b) * size_t(rows), workspace, as_stream(stream),
+                                                gemv_weights_static);
+    if (e != cudaSuccess) return MBOK_ERR_CUDA;
+  }
+  return MBOK_OK;
 }
 
 int mbok_gemv_set_static_weights(int on) {

@@ -266,15 +266,17 @@ __device__ __forceinline__ void prefetch_octet(const GemvParams& p, int slab, in
 // 128-column group) applied per lookup pair.  SV = true: the rank-1 form,
 // one kernel kk per CTA (K = 1 here; p.nk CTAs per slab), the tables built
 // from s_in^kk (.) x and each row's total scaled by s_out^kk[row].
+// The body of one CTA; `bid` is its index within the launch (or within its
+// matrix, for gemv_lut8_multi_kernel).
 template <int K, bool XF32, bool SV>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p) {
+__device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   using G = StageGeom<K>;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* tab = smem;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nvs = SV ? p.nslab * p.nk : p.nslab;   // (slab, kernel) CTAs per row range
-  const int vs = blockIdx.x % nvs, c = blockIdx.x / nvs;
+  const int vs = bid % nvs, c = bid / nvs;
   const int slab = SV ? vs % p.nslab : vs;
   const int kk = SV ? vs / p.nslab : 0;
   const int o_begin = int((long long)c * p.s.O / p.cps);
@@ -377,6 +379,61 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p
   cp_async_wait<0>();
   // With several CTAs per row range the partials are combined by
   // gemv_combine_kernel, launched right behind this grid.
+}
+
+template <int K, bool XF32, bool SV>
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_kernel(GemvParams p) {
+  gemv_lut8_body<K, XF32, SV>(p, int(blockIdx.x));
+}
+
+// Several matrices that share x (q/k/v, gate/up), each with its own K and
+// row count, in one launch: CTAs [cta0[s], cta0[s+1]) run matrix s with that
+// matrix's parameters (its own packed bits, scales, shape, output rows and
+// partial sums); K is a runtime switch per CTA.
+constexpr int kMaxSegments = 8;
+
+struct GemvMultiParams {
+  GemvParams seg[kMaxSegments];
+  int cta0[kMaxSegments + 1];
+  int nseg;
+};
+
+template <bool XF32>
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_multi_kernel(const __grid_constant__ GemvMultiParams mp) {
+  int sg = 0;
+  while (sg + 1 < mp.nseg && int(blockIdx.x) >= mp.cta0[sg + 1]) ++sg;
+  const GemvParams& p = mp.seg[sg];
+  const int bid = int(blockIdx.x) - mp.cta0[sg];
+  switch (p.s.K) {
+    case 1: gemv_lut8_body<1, XF32, false>(p, bid); break;
+    case 2: gemv_lut8_body<2, XF32, false>(p, bid); break;
+    case 3: gemv_lut8_body<3, XF32, false>(p, bid); break;
+    default: gemv_lut8_body<4, XF32, false>(p, bid); break;
+  }
+}
+
+struct CombineMultiParams {
+  const float* partial[kMaxSegments];   // matrix s: [nslab][O_s * 8]
+  int row0[kMaxSegments + 1];           // first output row of matrix s; row0[nseg] = total rows
+  int mpad[kMaxSegments];               // O_s * 8
+  int nseg, nvs;
+};
+
+// y[R] for the concatenated outputs: the matrix s that row R falls in, then
+// its slabs' partials in slab order (as gemv_combine_kernel).
+__global__ void __launch_bounds__(256) gemv_combine_multi_kernel(const __grid_constant__ CombineMultiParams cm,
+                                                                 float* __restrict__ y) {
+  allow_dependents();
+  grid_dependency_wait();
+  const int R = blockIdx.x * blockDim.x + threadIdx.x;
+  if (R >= cm.row0[cm.nseg]) return;
+  int sg = 0;
+  while (sg + 1 < cm.nseg && R >= cm.row0[sg + 1]) ++sg;
+  const int r = R - cm.row0[sg];
+  const float* part = cm.partial[sg];
+  float sum = 0.f;
+  for (int t = 0; t < cm.nvs; ++t) sum += __ldcg(part + size_t(t) * cm.mpad[sg] + r);
+  y[R] = sum;
 }
 
 // y[r] = sum over the nvs partials of row r, in (kernel, slab) order.  A
@@ -503,6 +560,104 @@ cudaError_t launch_gemv_lut(const uint8_t* packed, const uint16_t* alpha, const 
     case 8: return launch_k<4, false, false>(p, grid, stream);
     default: return launch_k<4, true, false>(p, grid, stream);
   }
+}
+
+// ---- several matrices sharing x in one launch ------------------------------
+
+// Partial sums of every matrix, one region per matrix: [nslab][O_s * 8].
+size_t gemv_multi_workspace_bytes(int nseg, const int* K, const int* M, int N) {
+  const size_t nslab = size_t((N + kSlabCols - 1) / kSlabCols);
+  if (nslab <= 1) return 0;
+  size_t total = 0;
+  for (int i = 0; i < nseg; ++i) total += nslab * size_t(make_shape(K[i], M[i], N).O) * kOctet * sizeof(float);
+  return total;
+}
+
+// y[0 .. sum M) = the matrices' outputs one after another, for one vector.
+// The row ranges per slab (cps) are shared out over the matrices by their
+// packed bytes (M_s * K_s), so one launch fills the SMs about as a single
+// matrix of the summed size would.
+cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const uint16_t* const* alpha, const int* K,
+                                  const int* M, int N, const void* x, bool x_f32, float* y, void* workspace,
+                                  cudaStream_t stream, bool weights_static) {
+  if (nseg < 1 || nseg > kMaxSegments) return cudaErrorInvalidValue;
+  const int sm = device_sm_count();
+  const int nslab = (N + kSlabCols - 1) / kSlabCols;
+  double wsum = 0.0;
+  for (int i = 0; i < nseg; ++i) wsum += double(M[i]) * K[i];
+  const int budget = sm / nslab > nseg ? sm / nslab : nseg;   // row ranges per slab, all matrices together
+  GemvMultiParams mp;
+  CombineMultiParams cm;
+  mp.nseg = cm.nseg = nseg;
+  cm.nvs = nslab;
+  int cta = 0, row = 0, max_k = 1;
+  size_t poff = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const Shape s = make_shape(K[i], M[i], N);
+    GemvParams& p = mp.seg[i];
+    p.packed = packed[i];
+    p.alpha = alpha[i];
+    p.s_in = nullptr;
+    p.s_out = nullptr;
+    p.x = x;
+    p.y = y + row;
+    p.s = s;
+    p.nslab = nslab;
+    int cps = int(double(budget) * double(M[i]) * K[i] / wsum);
+    if (cps < 1) cps = 1;
+    if (cps > s.O) cps = s.O;
+    p.cps = cps;
+    p.nk = 1;
+    p.weights_static = weights_static ? 1 : 0;
+    p.partial = nslab > 1 ? static_cast<float*>(workspace) + poff : nullptr;
+    mp.cta0[i] = cta;
+    cm.partial[i] = p.partial;
+    cm.row0[i] = row;
+    cm.mpad[i] = s.O * kOctet;
+    cta += nslab * cps;
+    row += M[i];
+    if (nslab > 1) poff += size_t(nslab) * s.O * kOctet;
+    if (K[i] > max_k) max_k = K[i];
+  }
+  mp.cta0[nseg] = cta;
+  cm.row0[nseg] = row;
+
+  auto fn = x_f32 ? gemv_lut8_multi_kernel<true> : gemv_lut8_multi_kernel<false>;
+  static bool attr_set[2] = {false, false};   // set once per variant, outside any stream capture
+  if (!attr_set[x_f32 ? 1 : 0]) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, StageGeom<4>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr_set[x_f32 ? 1 : 0] = true;
+  }
+  const int smem = max_k == 1 ? StageGeom<1>::kSmem
+                   : max_k == 2 ? StageGeom<2>::kSmem
+                   : max_k == 3 ? StageGeom<3>::kSmem
+                                : StageGeom<4>::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cta);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, mp);
+  if (e != cudaSuccess) return e;
+  if (nslab > 1) {
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3((row + 255) / 256);
+    c2.blockDim = dim3(256);
+    c2.stream = stream;
+    c2.attrs = attr;
+    c2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&c2, gemv_combine_multi_kernel, cm, y);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
 }
 
 // Rank-1 form: y = sum_k s_out^k (.) (B_k (s_in^k (.) x)) for one vector;

@@ -174,7 +174,10 @@ int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N
  * same K and N whose M are multiples of 8 concatenate along M by
  * concatenating their packed bytes and their blocked scales (both are
  * octet-major), and one mbok_gemv over the concatenation gives, row for row,
- * exactly the results of the separate calls (tested). */
+ * exactly the results of the separate calls (tested).  Matrices with
+ * different K (each layer's matrices may get their own number of kernels:
+ * Italian technical summary, 2D, kernel allocation) or any M fuse with
+ * mbok_gemv_multi below. */
 
 /* y[b][r] = sum_j W[r][j] * x[b][j] for b < batch (decode / small batch).
  * Evaluated as sum over groups and kernels of alpha[k][r][g] times the
@@ -219,6 +222,32 @@ size_t mbok_gemv_svid_workspace_bytes(int K, int M, int N, int batch);
 int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t* s_out, int K, int M, int N,
                    const void* x, int x_dtype, int batch, float* y, void* workspace, size_t workspace_bytes,
                    void* stream);
+
+/* Bytes of device workspace mbok_gemv_multi needs (same rules as
+ * mbok_gemv_workspace_bytes): the matrices' partial sums, one region per
+ * matrix.  0 if N <= 512 or on a bad argument. */
+size_t mbok_gemv_multi_workspace_bytes(int nseg, const int* K, const int* M, int N);
+
+/* Several matrices that read the same x, e.g. a layer's q, k and v or its
+ * gate and up projections, each with its own number of kernels K[s] and rows
+ * M[s], in one launch per vector:
+ *     y[b][R_s + r] = sum_j W_s[r][j] * x[b][j],   R_s = M[0] + ... + M[s-1],
+ * i.e. the matrices' outputs one after another in each output row of y
+ * (fp32 [batch][M[0] + ... + M[nseg-1]]).  The lookup-table kernel of
+ * mbok_gemv (any batch: one launch, plus the small launch that adds the
+ * slabs' partials, per vector); every output equals, bit for bit, that of
+ * mbok_gemv on the matrix alone with the lookup kernel (tested).
+ *   nseg       : 1..8 matrices.
+ *   packed[s], alpha[s] : matrix s in layout 1 with K[s] kernels (host arrays
+ *                of device pointers, each 16-byte aligned).
+ *   K[s], M[s] : host arrays; each (K[s], M[s], N) must be a valid shape and
+ *                the M[s] sum to at most 2^22.
+ *   N, group, x, x_dtype, batch, workspace, workspace_bytes, stream: as
+ *                mbok_gemv (workspace sized by mbok_gemv_multi_workspace_bytes).
+ * Calls sharing one workspace must not run concurrently. */
+int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* const* alpha, const int* K,
+                    const int* M, int N, int group, const void* x, int x_dtype, int batch, float* y,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Kernel choice of mbok_gemv and mbok_gemv_noalloc for this process (all
  * devices, all later calls):

@@ -186,3 +186,35 @@ def test_pointer_marshalling_checks_device(monkeypatch):
         mb._ptrs(Fake(1, contiguous=False))
     with pytest.raises(ValueError, match="CUDA tensors only"):
         mb.gemv(torch.zeros(4, dtype=torch.int32), None, 1, 8, 128, 128, None, mb.BF16, 1, None, None)
+
+
+def test_gemv_multi_sizes_and_argument_errors(L):
+    # mbok_gemv_multi: several matrices sharing x, each with its own K and M.
+    # Sizes and argument errors are host-side (nothing launches on an error).
+    import ctypes
+    import boolean_weight_matmul_b200 as mb
+    O = lambda M: (M + 7) // 8
+    # one region of [N/512 slabs][O_s * 8] fp32 partials per matrix
+    assert mb.gemv_multi_workspace_bytes([4, 2, 3], [5120, 136, 77], 5120) == \
+        10 * 4 * 8 * (O(5120) + O(136) + O(77))
+    assert mb.gemv_multi_workspace_bytes([4, 2], [64, 64], 512) == 0          # one slab: no workspace
+    assert mb.gemv_multi_workspace_bytes([5], [8], 1024) == 0                 # K out of range
+    assert mb.gemv_multi_workspace_bytes([1] * 9, [8] * 9, 1024) == 0         # more than 8 matrices
+    assert mb.gemv_multi_workspace_bytes([1, 1], [8, 1 << 22], 1024) == 0    # more than 2^22 rows in all
+
+    ia = lambda v: (ctypes.c_int * len(v))(*v)
+    dummy = (ctypes.c_void_p * 2)(0x1000, 0x2000)
+    call = lambda nseg, K, M, N=1024, group=128, dtype=1, batch=1, x=0x3000, y=0x4000: L.mbok_gemv_multi(
+        nseg, ctypes.cast(dummy, ctypes.c_void_p), ctypes.cast(dummy, ctypes.c_void_p),
+        ctypes.cast(ia(K), ctypes.c_void_p), ctypes.cast(ia(M), ctypes.c_void_p), N, group, x, dtype, batch, y,
+        None, 0, None)
+    assert call(0, [1], [8]) == 1                       # no matrix
+    assert call(9, [1] * 9, [8] * 9) == 1               # too many
+    assert call(2, [1, 5], [8, 8]) == 1                 # K out of range
+    assert call(2, [1, 2], [8, 0]) == 2                 # M < 1
+    assert call(2, [1, 2], [8, 8], N=1000) == 2         # N not a multiple of 128
+    assert call(2, [1, 2], [8, 8], group=64) == 4       # group != 128
+    assert call(2, [1, 2], [8, 8], dtype=7) == 1        # bad dtype
+    assert call(2, [1, 2], [8, 8], batch=17) == 1       # batch out of range
+    assert call(2, [1, 2], [8, 8], x=0x3008) == 3       # x not 16-byte aligned
+    assert call(2, [1, 2], [8, 8]) == 6                 # N > 512 needs a workspace

@@ -353,6 +353,52 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
 
 
+def _multi_case(Ks, Ms, N, batch, x_dtype, seed):
+    """mbok_gemv_multi over matrices with their own K and M, the separate
+    lookup-kernel calls, and the oracle (per matrix, concatenated)."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    signs = [wl.random_signs(K, M, N, seed + 10 * i) for i, (K, M) in enumerate(zip(Ks, Ms))]
+    alphas = [wl.alpha_decaying(K, M, N, seed + 10 * i + 1) for i, (K, M) in enumerate(zip(Ks, Ms))]
+    x = wl.x_normal(batch, N, seed + 99, x_dtype)
+    packed = [packed_from_signs_gpu(sg) for sg in signs]
+    alpha = [alpha_blocked_gpu(a, K, M, N) for a, K, M in zip(alphas, Ks, Ms)]
+    xd = x_dev(x, x_dtype)
+    dt = mb.F32 if x_dtype == "f32" else mb.BF16
+    y = torch.empty(batch, sum(Ms), dtype=torch.float32, device="cuda")
+    mb.gemv_multi(packed, alpha, Ks, Ms, N, 128, xd, dt, batch, y, mb.zeros_multi_workspace(Ks, Ms, N))
+    torch.cuda.synchronize()
+    with mb.gemv_kernel(mb.GEMV_LOOKUP):
+        sep = np.concatenate([gemv_gpu(p, a, K, M, N, x, x_dtype) for p, a, K, M in zip(packed, alpha, Ks, Ms)],
+                             axis=1)
+    refs = [O.linear(O.pack_signs(sg), a, K, M, N, x, x_dtype) for sg, a, K, M in zip(signs, alphas, Ks, Ms)]
+    y_ref = np.concatenate([r[0] for r in refs], axis=1)
+    E = np.concatenate([r[1] for r in refs], axis=1)
+    return y.cpu().numpy(), sep, y_ref, E
+
+
+@pytest.mark.parametrize("Ks,Ms,N,batch,x_dtype", [
+    ((4, 2, 3), (136, 64, 77), 1536, 1, "bf16"),     # mixed K, ragged M, 3 slabs
+    ((3, 1), (40, 8), 512, 2, "f32"),                 # one slab: outputs stored directly, two vectors
+    ((2,), (300,), 1024, 1, "bf16"),                  # a single matrix
+    ((1, 2, 3, 4, 1, 2, 3, 4), (8, 16, 24, 32, 40, 48, 56, 64), 640, 1, "bf16"),   # eight matrices, ragged slab
+])
+def test_gemv_multi_equals_separate_calls(Ks, Ms, N, batch, x_dtype):
+    # Each row is computed as in its own matrix's launch (same tables, same
+    # octet order, slabs added in order), so the fused outputs equal the
+    # separate lookup-kernel calls bit for bit, and the oracle within tolerance.
+    y, sep, y_ref, E = _multi_case(Ks, Ms, N, batch, x_dtype, 12000 + N + sum(Ms))
+    assert np.array_equal(y.view(np.uint32), sep.view(np.uint32))
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"multi K={Ks} M={Ms} N={N}")
+
+
+def test_gemv_multi_llama13b_qkv_mixed_k():
+    # LLaMA-13B q, k, v (5120 x 5120 each) with K = 4, 2, 3 in one launch.
+    y, sep, y_ref, E = _multi_case((4, 2, 3), (5120, 5120, 5120), 5120, 1, "bf16", 13000)
+    assert np.array_equal(y.view(np.uint32), sep.view(np.uint32))
+    assert_close(y, y_ref, E, GEMV_REL_L2, "13B qkv mixed K")
+
+
 def test_gemv_fused_projections_equal_separate_calls():
     # Matrices with the same K and N whose M are multiples of 8 fuse along M by
     # concatenating their packed bytes and blocked scales (octet-major storage):
