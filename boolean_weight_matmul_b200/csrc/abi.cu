@@ -1,6 +1,8 @@
 // C ABI of the MBOK library: argument checks on the host, then launches on
 // the caller's stream.  Nothing here allocates, synchronises or keeps state
 // beyond cached kernel attributes.
+#include <atomic>
+
 #include "mbok_common.cuh"
 
 namespace mbok {
@@ -34,25 +36,28 @@ cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const 
                            uint16_t*, cudaStream_t);
 unsigned gemm_error_flags();
 
-// Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc.
-int gemv_kernel_choice = MBOK_GEMV_AUTO;
+// Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc (atomic: host
+// threads may set and read it concurrently; a call reads it once).
+std::atomic<int> gemv_kernel_choice{MBOK_GEMV_AUTO};
 // Process-wide: GEMV weights may be read before the grid dependency wait
 // (see mbok_gemv_set_static_weights).
-bool gemv_weights_static = true;
+std::atomic<bool> gemv_weights_static{true};
 
 // One decode GEMV call: the lookup-table kernel once per vector, or the
 // tensor-core kernel over the whole batch.
 cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
                         bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
   bool tensor = batch > 1;
-  if (gemv_kernel_choice == MBOK_GEMV_LOOKUP) tensor = false;
-  if (gemv_kernel_choice == MBOK_GEMV_TENSOR) tensor = true;
+  const int choice = gemv_kernel_choice.load(std::memory_order_relaxed);
+  if (choice == MBOK_GEMV_LOOKUP) tensor = false;
+  if (choice == MBOK_GEMV_TENSOR) tensor = true;
+  const bool weights_static = gemv_weights_static.load(std::memory_order_relaxed);
   if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream);
   const size_t xbytes = x_f32 ? 4 : 2;
   for (int b = 0; b < batch; ++b) {
     const void* xb = static_cast<const char*>(x) + size_t(b) * s.N * xbytes;
     const cudaError_t e = launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream,
-                                          gemv_weights_static);
+                                          weights_static);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -249,7 +254,7 @@ int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* con
     const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
     const cudaError_t e = launch_gemv_lut_multi(nseg, p8, alpha, K, M, N, xb, x_dtype == MBOK_F32,
                                                 y + size_t(b) * size_t(rows), workspace, as_stream(stream),
-                                                gemv_weights_static);
+                                                gemv_weights_static.load(std::memory_order_relaxed));
     if (e != cudaSuccess) return MBOK_ERR_CUDA;
   }
   return MBOK_OK;
@@ -257,13 +262,13 @@ int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* con
 
 int mbok_gemv_set_static_weights(int on) {
   if (on != 0 && on != 1) return MBOK_ERR_INVALID_ARG;
-  gemv_weights_static = on == 1;
+  gemv_weights_static.store(on == 1, std::memory_order_relaxed);
   return MBOK_OK;
 }
 
 int mbok_gemv_set_kernel(int kernel) {
   if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TENSOR) return MBOK_ERR_INVALID_ARG;
-  gemv_kernel_choice = kernel;
+  gemv_kernel_choice.store(kernel, std::memory_order_relaxed);
   return MBOK_OK;
 }
 
@@ -292,7 +297,7 @@ int mbok_gemv_svid(const uint32_t* packed, const uint16_t* s_in, const uint16_t*
     const void* xb = static_cast<const char*>(x) + size_t(b) * N * xbytes;
     const cudaError_t e = launch_gemv_svid(reinterpret_cast<const uint8_t*>(packed), s_in, s_out, s, xb,
                                            x_dtype == MBOK_F32, y + size_t(b) * M, workspace, as_stream(stream),
-                                           gemv_weights_static);
+                                           gemv_weights_static.load(std::memory_order_relaxed));
     if (e != cudaSuccess) return MBOK_ERR_CUDA;
   }
   return MBOK_OK;

@@ -342,12 +342,9 @@ template <int K>
 static cudaError_t launch_tc_k(const CUtensorMap& xm, const CUtensorMap& bm, const CUtensorMap& am,
                                const TcParams& p, cudaStream_t stream) {
   auto fn = gemm_tc_kernel<K>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr_once;   // the attribute is per device context
+  const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), kTcSmem);
+  if (ae != cudaSuccess) return ae;
   const int tiles = ((p.s.M + kTcRows - 1) / kTcRows) * ((p.T + p.n_tile - 1) / p.n_tile);
   const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   fn<<<grid, kTcThreads, kTcSmem, stream>>>(xm, bm, am, p);

@@ -489,14 +489,9 @@ template <int K, bool XF32, bool SV>
 static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) {
   using G = StageGeom<K>;
   auto fn = gemv_lut8_kernel<K, XF32, SV>;
-  static bool attr_set = false;   // set once, outside any stream capture
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr_once;   // the attributes are per device context
+  const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), G::kSmem, true);
+  if (ae != cudaSuccess) return ae;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -623,14 +618,10 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
   cm.row0[nseg] = row;
 
   auto fn = x_f32 ? gemv_lut8_multi_kernel<true> : gemv_lut8_multi_kernel<false>;
-  static bool attr_set[2] = {false, false};   // set once per variant, outside any stream capture
-  if (!attr_set[x_f32 ? 1 : 0]) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, StageGeom<4>::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr_set[x_f32 ? 1 : 0] = true;
-  }
+  static PerDeviceOnce attr_once[2];   // per variant; the attributes are per device context
+  const cudaError_t ae = set_smem_attr_once(attr_once[x_f32 ? 1 : 0], reinterpret_cast<const void*>(fn),
+                                            StageGeom<4>::kSmem, true);
+  if (ae != cudaSuccess) return ae;
   const int smem = max_k == 1 ? StageGeom<1>::kSmem
                    : max_k == 2 ? StageGeom<2>::kSmem
                    : max_k == 3 ? StageGeom<3>::kSmem

@@ -557,12 +557,9 @@ template <int K, int NT, bool XF32, int MINB>
 static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
   auto fn = gemv_mma_kernel<K, NT, XF32, MINB>;
   using G = MmaGeom<K, NT, XF32>;
-  static bool attr_set = false;   // set once, outside any stream capture
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr_once;   // the attribute is per device context
+  const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), G::kSmem);
+  if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((p.s.O + 1) / 2);
   cfg.blockDim = dim3(kMmaThreads);

@@ -22,20 +22,19 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MBOK_NOALLOC_SC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
-
 // Set-up, once per device, with that device current: the device address of
-// the scratch array.  Returns nullptr if the runtime refuses.
+// the scratch array (cached per device index; host threads making their
+// first calls together at worst both look it up).  nullptr if the runtime
+// refuses.
 void* scratch_address() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (g_scratch_ptr[dev] == nullptr) {
+  static PerDeviceValue<void*> cache;
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  return cache.get(dev, []() -> void* {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+    return ptr;
+  });
 }
 
 }  // namespace

@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "../../include/mbok.h"
+#include "device_once.h"
 
 namespace mbok {
 
@@ -55,16 +56,34 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h2) {
   return __half22float2(h);
 }
 
-// SM count of the current device (queried once per process per device index).
+// The current device index, or -1 if the runtime cannot say.
+inline int current_device() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+// SM count of the current device (queried once per device index).
 inline int device_sm_count() {
-  static int cached[64] = {0};
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] > 0) return cached[dev];
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return 148;
-  cached[dev] = n;
-  return n;
+  static PerDeviceValue<int> cache;
+  const int dev = current_device();
+  const int n = cache.get(dev, [dev]() -> int {
+    int v = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return v > 0 ? v : 0;
+  });
+  return n > 0 ? n : 148;
+}
+
+// Dynamic shared-memory size (and, if asked, the largest shared-memory
+// carveout) of kernel `fn`, set once per device for the flag set `once`:
+// the runtime keeps these attributes per device context.
+inline cudaError_t set_smem_attr_once(PerDeviceOnce& once, const void* fn, int bytes, bool max_carveout = false) {
+  return static_cast<cudaError_t>(run_once_for_device(once, current_device(), [&]() -> int {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && max_carveout)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return static_cast<int>(e);
+  }));
 }
 
 }  // namespace mbok
