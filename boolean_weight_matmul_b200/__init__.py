@@ -25,6 +25,11 @@ MAX_BATCH = 16
 GEMV_AUTO = 0
 GEMV_LOOKUP = 1
 GEMV_TENSOR = 2
+GEMV_LOOKUP_SLABS = 3
+GEMV_LOOKUP_ROWS = 4
+GEMM_AUTO = 0
+GEMM_BF16 = 1
+GEMM_SPLIT = 2
 
 _lib = None
 
@@ -55,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "mbok_residual_binarize": ([vp, i, i, i, i, vp, vp, vp, vp], i),
             "mbok_gemv": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp], i),
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
+            "mbok_gemm_ex": ([vp, vp, i, i, i, i, vp, i, vp, i, vp], i),
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
             "mbok_check_wait_timeout": ([ctypes.c_uint, vp], i),
@@ -259,7 +265,7 @@ def gemv_noalloc(packed, alpha, K, M, N, group, x, x_dtype, batch, y, stream=Non
 
 def gemv_set_kernel(kernel: int) -> None:
     """Process-wide kernel choice of gemv / gemv_noalloc (GEMV_AUTO,
-    GEMV_LOOKUP or GEMV_TENSOR)."""
+    GEMV_LOOKUP, GEMV_TENSOR, GEMV_LOOKUP_SLABS or GEMV_LOOKUP_ROWS)."""
     _check(lib().mbok_gemv_set_kernel(kernel), "mbok_gemv_set_kernel")
 
 
@@ -285,9 +291,15 @@ class gemv_kernel:
         return False
 
 
-def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None) -> None:
+def gemm(packed, alpha, K, M, N, group, X, T, Y, stream=None, precision=None) -> None:
+    """mbok_gemm, or mbok_gemm_ex when a weight precision (GEMM_AUTO,
+    GEMM_BF16, GEMM_SPLIT) is given."""
     pp, pa, px, py = _ptrs(packed, alpha, X, Y)
-    _check(lib().mbok_gemm(pp, pa, K, M, N, group, px, T, py, _stream(stream)), "mbok_gemm")
+    if precision is None:
+        _check(lib().mbok_gemm(pp, pa, K, M, N, group, px, T, py, _stream(stream)), "mbok_gemm")
+    else:
+        _check(lib().mbok_gemm_ex(pp, pa, K, M, N, group, px, T, py, int(precision), _stream(stream)),
+               "mbok_gemm_ex")
 
 
 def read_device_errors() -> int:

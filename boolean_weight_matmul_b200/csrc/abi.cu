@@ -16,11 +16,14 @@ cudaError_t launch_svid_binarize(const float*, const Shape&, int, uint8_t*, __ha
                                  cudaStream_t);
 cudaError_t launch_gemv_lut(const uint8_t*, const uint16_t*, const Shape&, const void*, bool,
                             float*, void*, cudaStream_t, bool);
+cudaError_t launch_gemv_lut4(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, float*,
+                             cudaStream_t, bool);
+bool gemv_lut4_supported(const Shape&);
+unsigned gemv_lut4_error_flags();
 size_t gemv_lut_workspace_bytes(const Shape&);
 size_t gemv_svid_workspace_bytes(const Shape&);
 cudaError_t launch_gemv_svid(const uint8_t*, const uint16_t*, const uint16_t*, const Shape&, const void*, bool,
                              float*, void*, cudaStream_t, bool);
-unsigned gemv_error_flags();
 unsigned gemv_mma_error_flags();
 cudaError_t launch_wait_timeout_probe(unsigned, cudaStream_t);
 cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int,
@@ -33,7 +36,7 @@ cudaError_t launch_gemv_lut_multi(int, const uint8_t* const*, const uint16_t* co
 size_t gemv_multi_workspace_bytes(int, const int*, const int*, int);
 
 cudaError_t launch_gemm_tc(const uint8_t*, const uint16_t*, const Shape&, const uint16_t*, int,
-                           uint16_t*, cudaStream_t);
+                           uint16_t*, bool, cudaStream_t);
 unsigned gemm_error_flags();
 
 // Process-wide kernel choice of mbok_gemv / mbok_gemv_noalloc (atomic: host
@@ -43,21 +46,28 @@ std::atomic<int> gemv_kernel_choice{MBOK_GEMV_AUTO};
 // (see mbok_gemv_set_static_weights).
 std::atomic<bool> gemv_weights_static{true};
 
-// One decode GEMV call: the lookup-table kernel once per vector, or the
-// tensor-core kernel over the whole batch.
+// One decode GEMV call: a lookup-table kernel once per vector -- 512-column
+// slabs with 8-bit tables and a combine launch, or, when asked for, whole rows
+// with 4-bit tables in one launch where they fit one CTA (N <= 10240) -- or
+// the tensor-core kernel over the whole batch.
 cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
                         bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
   bool tensor = batch > 1;
   const int choice = gemv_kernel_choice.load(std::memory_order_relaxed);
-  if (choice == MBOK_GEMV_LOOKUP) tensor = false;
+  if (choice == MBOK_GEMV_LOOKUP || choice == MBOK_GEMV_LOOKUP_SLABS || choice == MBOK_GEMV_LOOKUP_ROWS)
+    tensor = false;
   if (choice == MBOK_GEMV_TENSOR) tensor = true;
   const bool weights_static = gemv_weights_static.load(std::memory_order_relaxed);
   if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream);
+  // Whole rows only when asked for: on B200 the slab kernel is measured
+  // faster on the LLaMA shapes (see the design notes).
+  const bool rows = choice == MBOK_GEMV_LOOKUP_ROWS && gemv_lut4_supported(s);
   const size_t xbytes = x_f32 ? 4 : 2;
   for (int b = 0; b < batch; ++b) {
     const void* xb = static_cast<const char*>(x) + size_t(b) * s.N * xbytes;
-    const cudaError_t e = launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream,
-                                          weights_static);
+    const cudaError_t e =
+        rows ? launch_gemv_lut4(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, stream, weights_static)
+             : launch_gemv_lut(packed, alpha, s, xb, x_f32, y + size_t(b) * s.M, workspace, stream, weights_static);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -267,7 +277,7 @@ int mbok_gemv_set_static_weights(int on) {
 }
 
 int mbok_gemv_set_kernel(int kernel) {
-  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_TENSOR) return MBOK_ERR_INVALID_ARG;
+  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_LOOKUP_ROWS) return MBOK_ERR_INVALID_ARG;
   gemv_kernel_choice.store(kernel, std::memory_order_relaxed);
   return MBOK_OK;
 }
@@ -311,7 +321,7 @@ int mbok_check_wait_timeout(unsigned timeout_us, void* stream) {
 int mbok_read_device_errors(unsigned* flags) {
   if (flags == nullptr) return MBOK_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return MBOK_ERR_CUDA;
-  const unsigned g = gemv_error_flags();
+  const unsigned g = gemv_lut4_error_flags();
   const unsigned m = gemm_error_flags();
   const unsigned t = gemv_mma_error_flags();
   if (g == ~0u || m == ~0u || t == ~0u) return MBOK_ERR_CUDA;
@@ -319,18 +329,25 @@ int mbok_read_device_errors(unsigned* flags) {
   return MBOK_OK;
 }
 
-int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
-              const uint16_t* X, int T, uint16_t* Y, void* stream) {
+int mbok_gemm_ex(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+                 const uint16_t* X, int T, uint16_t* Y, int precision, void* stream) {
   const int st = check_shape(K, M, N);
   if (st != MBOK_OK) return st;
   if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
   if (T < 1 || T > (1 << 23)) return MBOK_ERR_SHAPE;
   if (packed == nullptr || alpha == nullptr || X == nullptr || Y == nullptr)
     return MBOK_ERR_INVALID_ARG;
+  if (precision < MBOK_GEMM_AUTO || precision > MBOK_GEMM_SPLIT) return MBOK_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(X, 16) || !aligned(Y, 16))
     return MBOK_ERR_ALIGN;
+  const bool split = precision == MBOK_GEMM_SPLIT || (precision == MBOK_GEMM_AUTO && N <= MBOK_GEMM_SPLIT_MAX_N);
   return from_cuda(launch_gemm_tc(reinterpret_cast<const uint8_t*>(packed), alpha, make_shape(K, M, N), X,
-                                  T, Y, as_stream(stream)));
+                                  T, Y, split, as_stream(stream)));
+}
+
+int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const uint16_t* X, int T, uint16_t* Y, void* stream) {
+  return mbok_gemm_ex(packed, alpha, K, M, N, group, X, T, Y, MBOK_GEMM_AUTO, stream);
 }
 
 }  // extern "C"

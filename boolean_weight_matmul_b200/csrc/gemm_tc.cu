@@ -17,11 +17,10 @@
 //     128-byte swizzle; the tile's packed bits (16 octets x K x 64 bytes) and
 //     scales (16 octets x K x 8 fp16) come with two more TMA loads (warp 0);
 //   * W tile, 256 rows x 64 columns bf16 (32 KB): written by 16 unpack warps
-//     (two rows x 16 columns per thread) in the same swizzled K-major layout.  For a column pair (2i, 2i+1) of a row
-//     the two sign bits are brought to bit 15 and bit 31 by one shift of
-//     (h | h << 15), where h holds the row's 16 bits of one kernel, and
-//     applied to the bf16 scale pair with one LOP3; the K kernels are summed
-//     with packed bf16 adds (HADD2);
+//     (two rows x 16 columns per thread) in the same swizzled K-major layout;
+//     each element is its weight level rounded once to bf16, selected from
+//     the 2^K levels of its (row, group) by its K bits (see the unpack
+//     section below);
 //   * one thread (warp 1) issues 2 x 4 tcgen05.mma (M=128, N=n, K=16), one
 //     set per row half, into the tensor-memory accumulators and commits them
 //     to the stage's "empty" barrier.
@@ -39,18 +38,27 @@ constexpr int kTcRows = 256;      // weight rows per CTA: two M=128 MMAs share e
 constexpr int kTcHalf = 128;      // MMA M
 constexpr int kTcTokens = 256;    // largest token tile per CTA (MMA N); the host picks <= this
 constexpr int kTcBK = 64;         // columns per stage (one 128-byte swizzle row)
-constexpr int kTcStages = 3;
 constexpr int kTcXBytes = kTcTokens * kTcBK * 2;   // 32 KB
 constexpr int kTcWBytes = kTcRows * kTcBK * 2;     // 32 KB (two 16 KB halves)
 constexpr int kTcOctets = kTcRows / kOctet;        // 32 row octets per tile
 constexpr int kTcBitsRow = kTcBK / 8;              // 64 columns = 8 bytes per row = 64 bytes per octet
 constexpr int kTcBitsBytes = kTcOctets * MBOK_MAX_K * kTcBitsRow * kOctet;   // 8 KB (K = 4)
 constexpr int kTcAlphaBytes = kTcOctets * MBOK_MAX_K * 16;                 // 2 KB (K = 4)
-constexpr int kTcStageBytes = kTcXBytes + kTcWBytes + kTcBitsBytes + kTcAlphaBytes;
+// One stage: X tile, the W tile (two tiles, hi and lo, when each weight is
+// split into two bf16 terms), the packed bits and the scales.  Three stages,
+// or two with the split.
+template <bool SPLIT>
+struct TcGeom {
+  static constexpr int kStages = SPLIT ? 2 : 3;
+  static constexpr int kWTiles = SPLIT ? 2 : 1;
+  static constexpr int kBitsOff = kTcXBytes + kWTiles * kTcWBytes;
+  static constexpr int kAlphaOff = kBitsOff + kTcBitsBytes;
+  static constexpr int kStageBytes = kAlphaOff + kTcAlphaBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;   // + alignment + barriers
+};
 constexpr int kTcUnpackWarps = 16;
 constexpr int kTcEpiWarp0 = 2 + kTcUnpackWarps;                 // 4 epilogue warps follow the unpack warps
 constexpr int kTcThreads = (2 + kTcUnpackWarps + 4) * 32;       // TMA, MMA, 16 unpack, 4 epilogue
-constexpr int kTcSmem = kTcStages * kTcStageBytes + 1024 + 256;  // + alignment + barriers
 constexpr unsigned kTcTmemCols = 512;      // row halves 0 and 1: columns 0.. and 256..
 
 // Instruction descriptor: D f32, A bf16, B bf16, both K-major, M=128, N=n.
@@ -69,85 +77,214 @@ struct TcParams {
 };
 
 // ---------------------------------------------------------------------------
-// Unpack: 2 rows x 16 columns of W (all K kernels) -> bf16 in the swizzled tile
+// Unpack: one row x 16 columns of W (all K kernels) -> bf16 in the swizzled tile
 // ---------------------------------------------------------------------------
+//
+// An element of the tile is the weight level its K bits select, rounded once:
+//     Wt[r][j] = RN_bf16( s_0 a_0 + s_1 a_1 + ... + s_{K-1} a_{K-1} ),
+// s_k = +1 for a set bit and -1 for a clear one, a_k the fp16 group scales,
+// the sum taken in fp32 in kernel order.  K kernels give at most 2^K levels
+// per (row, group) (Paper-Notes page, 关键设计: K Boolean kernels represent
+// 2^K weight values), so each level is formed once per (row, group) and the
+// per-element work is a selection:
+//  * K = 1: the level is +-a_0; one LOP3 applies the sign bit pair.
+//  * K = 2: the four levels sit in two registers as bf16; a byte permute
+//    (PRMT) whose selector is built from the two bits of each element picks
+//    an element pair's levels at once.
+//  * K = 3, 4: the levels are sign-symmetric (the level of the complemented
+//    bits is the negated level, exactly, since rounding to nearest is
+//    symmetric), so only the 2^(K-1) levels with s_0 = +1 are kept: the other
+//    bits are replaced by t_k = XNOR(b_k, b_0), a PRMT (two and a select for
+//    K = 4) picks M[t], and the sign of b_0 is applied with one LOP3.
+// The PRMT selector of columns (2p, 2p+1) needs 2*index in both nibbles of
+// each output halfword; index bits sit in a precomputed word Z at 2p+1,
+// 2p+2 (column 2p) and 2p+9, 2p+10 (column 2p+1), so the selector is
+// ((Z >> 2p) & 0x0606) * 0x11 + 0x1010.
 
-// Sign-applied scale pair for columns (2i, 2i+1): the scale's sign flips
-// where the bit is 0 (-1).  u = h | (h << 15) holds bit b at b and at 15 + b,
-// so one left shift by 15 - 2i puts bit 2i at 15 and bit 2i+1 at 31.
-template <int I>
-__device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t a2) {
-  const uint32_t s = u << (15 - 2 * I);
+// bf16 pair (lo, hi), each rounded to nearest even from fp32.
+__device__ __forceinline__ uint32_t tc_pack_bf16x2(float lo, float hi) {
   uint32_t r;
-  // r = (~s & 0x80008000) ^ a2
-  asm("lop3.b32 %0, %1, %2, %3, 0xA6;\n" : "=r"(r) : "r"(s), "r"(0x80008000u), "r"(a2));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 
-__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
-  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
-  __nv_bfloat162 z = __hadd2(x, y);
-  return *reinterpret_cast<uint32_t*>(&z);
+// Sign-applied level pair for columns (2i, 2i+1): the level's sign flips
+// where the bit of kernel 0 is 0.  u = h | (h << 15) holds bit b at b and at
+// 15 + b, so one left shift by 15 - 2i puts bit 2i at 15 and bit 2i+1 at 31.
+template <int I>
+__device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t lev) {
+  const uint32_t s = u << (15 - 2 * I);
+  uint32_t r;
+  // r = (~s & 0x80008000) ^ lev
+  asm("lop3.b32 %0, %1, %2, %3, 0xA6;\n" : "=r"(r) : "r"(s), "r"(0x80008000u), "r"(lev));
+  return r;
 }
 
+// Index words of 16 columns from two 16-bit planes (A: index bit 0, B:
+// index bit 1): z[0] covers columns 0..7, z[1] columns 8..15 (layout above).
+__device__ __forceinline__ void tc_index_words(uint32_t A, uint32_t B, uint32_t z[2]) {
+  z[0] = ((A & 0x55u) << 1) | ((A & 0xAAu) << 8) | ((B & 0x55u) << 2) | ((B & 0xAAu) << 9);
+  z[1] = ((A & 0x5500u) >> 7) | (A & 0xAA00u) | ((B & 0x5500u) >> 6) | ((B & 0xAA00u) << 1);
+}
+
+// prmt.b32 in its default mode, where bit 3 of a selector nibble replicates
+// the sign (bit 7) of the selected byte (the __byte_perm intrinsic only
+// honours the low three bits of each nibble).
+__device__ __forceinline__ uint32_t tc_prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// PRMT selector for column pair I from the index words.
+template <int I>
+__device__ __forceinline__ uint32_t tc_selector(const uint32_t z[2]) {
+  const uint32_t v = (z[I >> 2] >> (2 * (I & 3))) & 0x0606u;
+  return v * 0x11u + 0x1010u;
+}
+
+// Levels of one (row, group) from its K fp16 scales (kernel order), as fp32:
+//   K = 1: v = {a0};
+//   K = 2: v = {V0, V1, V2, V3}, V[b0 + 2 b1] = s0 a0 + s1 a1;
+//   K = 3: v = {M0 .. M3}, M[t1 + 2 t2] = (a0 + s1 a1) + s2 a2;
+//   K = 4: v = {M0 .. M7}, M[t1 + 2 t2 + 4 t3] = ((a0 + s1 a1) + s2 a2) + s3 a3.
 template <int K>
-__device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_t a2[K], uint32_t out[8]) {
-  uint32_t u[K];
+__device__ __forceinline__ void tc_level_values(const unsigned char* alpha, int o, int i, float v[8]) {
+  float a[K];
 #pragma unroll
-  for (int k = 0; k < K; ++k) u[k] = h[k] | (h[k] << 15);
-#define MBOK_PAIR(I)                                                     \
-  {                                                                      \
-    uint32_t v = tc_signed_pair<I>(u[0], a2[0]);                         \
-    _Pragma("unroll") for (int k = 1; k < K; ++k) v = bf16x2_add(v, tc_signed_pair<I>(u[k], a2[k])); \
-    out[I] = v;                                                          \
+  for (int k = 0; k < K; ++k)
+    a[k] = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(alpha + (o * K + k) * 16 + 2 * i)));
+  if (K == 1) {
+    v[0] = a[0];
+  } else if (K == 2) {
+    const float d = a[0] - a[1], e = a[0] + a[1];
+    v[0] = -e; v[1] = d; v[2] = -d; v[3] = e;
+  } else {
+    const float x = a[0] - a[1], y = a[0] + a[1];
+    const float a2 = a[K > 2 ? 2 : 0];
+    const float c0 = x - a2, c1 = y - a2, c2 = x + a2, c3 = y + a2;
+    if (K == 3) {
+      v[0] = c0; v[1] = c1; v[2] = c2; v[3] = c3;
+    } else {
+      const float a3 = a[K > 3 ? 3 : 0];
+      v[0] = c0 - a3; v[1] = c1 - a3; v[2] = c2 - a3; v[3] = c3 - a3;
+      v[4] = c0 + a3; v[5] = c1 + a3; v[6] = c2 + a3; v[7] = c3 + a3;
+    }
   }
-  MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
-#undef MBOK_PAIR
 }
 
-// bf16 pair (a, a) from an fp16 scale.
-__device__ __forceinline__ uint32_t tc_scale_pair(uint32_t h16) {
-  const float a = __half2float(__ushort_as_half(uint16_t(h16)));
-  const __nv_bfloat16 b = __float2bfloat16_rn(a);
-  const uint32_t bb = __bfloat16_as_ushort(b);
-  return bb | (bb << 16);
+// The level registers of one (row, group): P holds the levels rounded once
+// to bf16 (low half first; K = 1: (a0, a0)), and, for the split, L holds
+// what that rounding left, v - RN_bf16(v) (exact in fp32), rounded to bf16.
+// Rounding to nearest is sign-symmetric, so both stay exact negations of the
+// complemented levels.
+template <int K, bool SPLIT>
+__device__ __forceinline__ void tc_levels(const unsigned char* alpha, int o, int i, uint32_t P[4], uint32_t L[4]) {
+  float v[8];
+  tc_level_values<K>(alpha, o, i, v);
+  constexpr int kN = K == 1 ? 1 : (K == 4 ? 8 : 4);
+  float hi[8], lo[8];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) {
+    hi[n] = __bfloat162float(__float2bfloat16_rn(v[n]));
+    lo[n] = v[n] - hi[n];
+  }
+  if (K == 1) {
+    P[0] = tc_pack_bf16x2(hi[0], hi[0]);
+    if (SPLIT) L[0] = tc_pack_bf16x2(lo[0], lo[0]);
+  } else {
+#pragma unroll
+    for (int n = 0; n < kN / 2; ++n) {
+      P[n] = tc_pack_bf16x2(hi[2 * n], hi[2 * n + 1]);
+      if (SPLIT) L[n] = tc_pack_bf16x2(lo[2 * n], lo[2 * n + 1]);
+    }
+  }
+}
+
+// One row x 16 columns: h[k] = the row's 16 bits of kernel k (column b in
+// bit b), P = its levels; out[I] = bf16 pair of columns (2I, 2I+1).
+template <int K>
+__device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_t P[4], uint32_t out[8]) {
+  const uint32_t u0 = h[0] | (h[0] << 15);
+  if (K == 1) {
+#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, P[0]);
+    MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
+#undef MBOK_PAIR
+  } else if (K == 2) {
+    uint32_t z[2];
+    tc_index_words(h[0], h[1], z);
+#define MBOK_PAIR(I) out[I] = __byte_perm(P[0], P[1], tc_selector<I>(z));
+    MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
+#undef MBOK_PAIR
+  } else {
+    // t_k = XNOR(b_k, b_0): the bits relative to kernel 0 (only bits 0..15 are read)
+    const uint32_t t1 = ~(h[1] ^ h[0]), t2 = ~(h[2 % K] ^ h[0]);
+    uint32_t z[2];
+    tc_index_words(t1, t2, z);
+    if (K == 3) {
+#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, __byte_perm(P[0], P[1], tc_selector<I>(z)));
+      MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
+#undef MBOK_PAIR
+    } else {
+      const uint32_t t3 = ~(h[3 % K] ^ h[0]) & 0xFFFFu;
+      const uint32_t u3 = t3 | (t3 << 15);
+      // 16-bit masks from bit 15 / bit 31 of the shifted t3 word (sign-replicating permute)
+#define MBOK_PAIR(I)                                                           \
+  {                                                                            \
+    const uint32_t sel = tc_selector<I>(z);                                    \
+    const uint32_t lo = __byte_perm(P[0], P[1], sel);                          \
+    const uint32_t hi = __byte_perm(P[2], P[3], sel);                          \
+    const uint32_t m = tc_prmt(u3 << (15 - 2 * I), 0u, 0xBB99u);               \
+    out[I] = tc_signed_pair<I>(u0, (hi & m) | (lo & ~m));                      \
+  }
+      MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
+#undef MBOK_PAIR
+    }
+  }
 }
 
 // Unpack one row x 16 columns: thread tid -> row r = tid >> 2, unit u = tid & 3
-// of the 128 x 64 tile.  Bits and scales come from the stage's TMA-loaded
-// copies: bits [octet][k][unit][row] halfwords, scales [octet][k][row] fp16.
-template <int K>
-__device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, const unsigned char* alpha,
-                                                    unsigned char* wtile, int tid) {
+// of the 256 x 64 tile, with the row's levels P for the stage's group.  Bits
+// come from the stage's TMA-loaded copy, [octet][k][unit][row] halfwords.
+template <int K, bool SPLIT>
+__device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, const uint32_t P[4],
+                                                    const uint32_t L[4], unsigned char* wtile, int tid) {
   const int r = tid >> 2, u = tid & 3;
   const int o = r >> 3, i = r & 7;
-  uint32_t h[K], a2[K], out[8];
+  uint32_t h[K], out[8];
 #pragma unroll
-  for (int k = 0; k < K; ++k) {
+  for (int k = 0; k < K; ++k)
     h[k] = *reinterpret_cast<const uint16_t*>(bits + ((o * K + k) * 4 + u) * 16 + 2 * i);
-    a2[k] = tc_scale_pair(*reinterpret_cast<const uint16_t*>(alpha + (o * K + k) * 16 + 2 * i));
-  }
-  tc_unpack_row<K>(h, a2, out);
   // 16 columns = chunks 2u and 2u+1 of the row's 128-byte line, swizzled; the
   // 8 threads of a store phase hold 2 rows of opposite parity x 4 units, i.e.
   // 8 distinct chunks.
-  unsigned char* line = wtile + r * 128;
   const int c0 = (2 * u) ^ (r & 7), c1 = (2 * u + 1) ^ (r & 7);
+  tc_unpack_row<K>(h, P, out);
+  unsigned char* line = wtile + r * 128;
   *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
   *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
+  if (SPLIT) {
+    // the same selection from the residual levels, into the second tile
+    tc_unpack_row<K>(h, L, out);
+    line += kTcWBytes;
+    *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
+  }
 }
 
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
 
-template <int K>
+template <int K, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
                const __grid_constant__ CUtensorMap amap, TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using G = TcGeom<SPLIT>;
+  constexpr int kTcStages = G::kStages;
+  constexpr int kTcStageBytes = G::kStageBytes;
   uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // stage's TMA data landed
   uint64_t* full_w = full_x + kTcStages;   // stage's W tile unpacked
   uint64_t* empty = full_w + kTcStages;    // stage's MMAs done
@@ -200,8 +337,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
           unsigned char* st = smem + s * kTcStageBytes;
           tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2 + kTcOctets * K * (kTcBitsRow * kOctet + 16));
           tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
-          tc_tma_load_2d(st + kTcXBytes + kTcWBytes, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
-          tc_tma_load_2d(st + kTcXBytes + kTcWBytes + kTcBitsBytes, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
+          tc_tma_load_2d(st + G::kBitsOff, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
+          tc_tma_load_2d(st + G::kAlphaOff, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
                          r0 / kOctet, &full_x[s]);
         }
       }
@@ -224,9 +361,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
           for (int kk = 0; kk < kTcBK / 16; ++kk) {
             const uint64_t bdesc = tc_desc_sw128(xs + kk * 32);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < 2; ++h) {
               tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + h * (kTcHalf * 128) + kk * 32), bdesc, p.idesc,
                      (kb > 0 || kk > 0) ? 1u : 0u);
+              if (SPLIT)   // the residual tile into the same accumulator
+                tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + kTcWBytes + h * (kTcHalf * 128) + kk * 32), bdesc,
+                       p.idesc, 1u);
+            }
           }
           tc_commit(&empty[s]);
         }
@@ -237,6 +378,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   } else if (warp < kTcEpiWarp0) {
     // ---- unpack warps ----
     const int tid = threadIdx.x - 64;
+    uint32_t lev[2][4] = {}, res[2][4] = {};   // this thread's two rows' levels for the current group
     int g = 0;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -244,10 +386,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         // the stage's TMA loads landing also means its previous MMAs are done
         if (!tc_wait(&full_x[s], unsigned(g / kTcStages) & 1u)) { ok = false; break; }
         unsigned char* st = smem + s * kTcStageBytes;
+        // a 128-column group spans two 64-column stages: its levels are
+        // formed on the first and kept for the second
+        if ((kb & 1) == 0) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int r = (tid + j * kTcUnpackWarps * 32) >> 2;
+            tc_levels<K, SPLIT>(st + G::kAlphaOff, r >> 3, r & 7, lev[j], res[j]);
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          tc_unpack_from_smem<K>(st + kTcXBytes + kTcWBytes, st + kTcXBytes + kTcWBytes + kTcBitsBytes,
-                                 st + kTcXBytes, tid + j * kTcUnpackWarps * 32);
+          tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], st + kTcXBytes,
+                                        tid + j * kTcUnpackWarps * 32);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
         tc_arrive(&full_w[s]);
       }
@@ -338,10 +489,11 @@ unsigned gemm_error_flags() {
   return v;
 }
 
-template <int K>
+template <int K, bool SPLIT>
 static cudaError_t launch_tc_k(const CUtensorMap& xm, const CUtensorMap& bm, const CUtensorMap& am,
                                const TcParams& p, cudaStream_t stream) {
-  auto fn = gemm_tc_kernel<K>;
+  auto fn = gemm_tc_kernel<K, SPLIT>;
+  constexpr int kTcSmem = TcGeom<SPLIT>::kSmem;
   static PerDeviceOnce attr_once;   // the attribute is per device context
   const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), kTcSmem);
   if (ae != cudaSuccess) return ae;
@@ -370,9 +522,10 @@ int tc_token_tile(int M, int T, int sms) {
   return best;
 }
 
-// Returns cudaErrorNotSupported when the tensor-map encoder is unavailable.
+// split: each weight as two bf16 terms (see the header).  Returns
+// cudaErrorNotSupported when the tensor-map encoder is unavailable.
 cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const uint16_t* X,
-                           int T, uint16_t* Y, cudaStream_t stream) {
+                           int T, uint16_t* Y, bool split, cudaStream_t stream) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   const int n_tile = tc_token_tile(s.M, T, device_sm_count());
@@ -414,10 +567,10 @@ cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const S
   p.n_tile = n_tile;
   p.idesc = tc_idesc(n_tile);
   switch (s.K) {
-    case 1: return launch_tc_k<1>(xm, bm, am, p, stream);
-    case 2: return launch_tc_k<2>(xm, bm, am, p, stream);
-    case 3: return launch_tc_k<3>(xm, bm, am, p, stream);
-    default: return launch_tc_k<4>(xm, bm, am, p, stream);
+    case 1: return split ? launch_tc_k<1, true>(xm, bm, am, p, stream) : launch_tc_k<1, false>(xm, bm, am, p, stream);
+    case 2: return split ? launch_tc_k<2, true>(xm, bm, am, p, stream) : launch_tc_k<2, false>(xm, bm, am, p, stream);
+    case 3: return split ? launch_tc_k<3, true>(xm, bm, am, p, stream) : launch_tc_k<3, false>(xm, bm, am, p, stream);
+    default: return split ? launch_tc_k<4, true>(xm, bm, am, p, stream) : launch_tc_k<4, false>(xm, bm, am, p, stream);
   }
 }
 

@@ -71,6 +71,8 @@ typedef enum { MBOK_F32 = 0, MBOK_BF16 = 1 } mbok_dtype;
 #define MBOK_GEMV_AUTO 0
 #define MBOK_GEMV_LOOKUP 1
 #define MBOK_GEMV_TENSOR 2
+#define MBOK_GEMV_LOOKUP_SLABS 3
+#define MBOK_GEMV_LOOKUP_ROWS 4
 /* Size of the scratch array built into the library for mbok_gemv_noalloc. */
 #define MBOK_NOALLOC_SCRATCH_BYTES (4u << 20)
 
@@ -86,12 +88,13 @@ size_t mbok_packed_bytes(int K, int M, int N);
 /* fp16 elements of the blocked scales: ceil(M/8)*8*(N/128)*K.  0 on bad shape. */
 size_t mbok_alpha_elems(int K, int M, int N);
 
-/* Bytes of device workspace mbok_gemv needs for (K, M, N, batch).  The caller
- * allocates it (256-byte aligned; no initialisation needed) and may reuse it
- * for any later call with the same or smaller requirement.  It holds the
- * per-CTA partial sums of one call, which a second, small launch of the same
- * call adds up in a fixed order.  Calls that share one workspace must not run
- * concurrently (calls in one stream are fine). */
+/* Bytes of device workspace mbok_gemv needs for (K, M, N, batch), whichever
+ * kernel the call takes.  The caller allocates it (256-byte aligned; no
+ * initialisation needed) and may reuse it for any later call with the same or
+ * smaller requirement.  Only the 8-bit slab lookup kernel uses it: it holds
+ * the per-CTA partial sums of one call, which a second, small launch of the
+ * same call adds up in a fixed order.  Calls that share one workspace must
+ * not run concurrently (calls in one stream are fine). */
 size_t mbok_gemv_workspace_bytes(int K, int M, int N, int batch);
 
 /* Pack K sign matrices into layout 1.
@@ -253,12 +256,16 @@ int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* con
  * devices, all later calls):
  *   MBOK_GEMV_AUTO (default): lookup tables for one vector, tensor cores for
  *     more;
- *   MBOK_GEMV_LOOKUP: lookup tables (8-bit tables over 512-column slabs;
- *     the slabs' partial sums are added by a second small launch through the
- *     workspace), once per vector;
- *   MBOK_GEMV_TENSOR: tensor cores for any batch.
- * Both kernels meet the accuracy stated for mbok_gemv; results differ in
- * rounding.  Not synchronised with calls in flight on other host threads.
+ *   MBOK_GEMV_LOOKUP: lookup tables, once per vector: 8-bit tables over
+ *     512-column slabs, whose partial sums a second small launch adds
+ *     through the workspace;
+ *   MBOK_GEMV_TENSOR: tensor cores for any batch;
+ *   MBOK_GEMV_LOOKUP_SLABS: the slab lookup kernel (as MBOK_GEMV_LOOKUP);
+ *   MBOK_GEMV_LOOKUP_ROWS: whole rows per CTA with 4-bit tables, one launch
+ *     and no workspace, where those tables fit one CTA's shared memory
+ *     (N <= 10240; wider rows take the slab kernel).
+ * All kernels meet the accuracy stated for mbok_gemv; results differ in
+ * rounding.  Atomic, but calls already issued keep the kernel they chose.
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);
 
@@ -287,10 +294,12 @@ int mbok_gemv_set_static_weights(int on);
  * property of the library, not of the method.)
  *
  * Same arguments, results and accuracy as mbok_gemv, minus the workspace.
- * The scratch mbok_gemv would take from the workspace comes instead from one
- * array of MBOK_NOALLOC_SCRATCH_BYTES (4 MiB) compiled into the library; every
- * GPU that loads the library holds that array until the process exits.  This
- * entry point calls no allocating routine (no cudaMalloc / cudaFree).
+ * The scratch mbok_gemv would take from the workspace (the partial sums of
+ * the 8-bit slab lookup kernel; the whole-row lookup and tensor-core kernels
+ * need none) comes instead from one array of MBOK_NOALLOC_SCRATCH_BYTES
+ * (4 MiB) compiled into the library; every GPU that loads the library holds
+ * that array until the process exits.  This entry point calls no allocating
+ * routine (no cudaMalloc / cudaFree).
  *  - Limit: shapes whose mbok_gemv_workspace_bytes exceeds
  *    MBOK_NOALLOC_SCRATCH_BYTES are rejected with MBOK_ERR_SCRATCH_LIMIT
  *    (roughly M * N > 500 million weights).
@@ -308,11 +317,11 @@ int mbok_gemv_noalloc(const uint32_t* packed, const uint16_t* alpha, int K, int 
 /* Diagnostic: waits inside the library's kernels are bounded (about a second);
  * a kernel that gives up records a flag and returns early instead of hanging.
  * Writes the flags accumulated on the current device since the last call to
- * *flags (0 = none; bit 1 = a prefill-GEMM pipeline wait gave up; bit 2 = a
- * tensor-core GEMV copy wait gave up, in which case that launch stored no
- * outputs; bit 0 is reserved and stays 0: the lookup-table GEMV never waits)
- * and clears them.  Synchronises the device.  Returns MBOK_ERR_CUDA if the
- * flags cannot be read. */
+ * *flags (0 = none; bit 0 = a whole-row lookup GEMV copy wait gave up, in
+ * which case that CTA stored none of its rows of y; bit 1 = a prefill-GEMM
+ * pipeline wait gave up; bit 2 = a tensor-core GEMV copy wait gave up, in
+ * which case that launch stored no outputs) and clears them.  Synchronises
+ * the device.  Returns MBOK_ERR_CUDA if the flags cannot be read. */
 int mbok_read_device_errors(unsigned* flags);
 
 /* Self-check of the bounded waits that the pipelined kernels use: launches
@@ -322,20 +331,36 @@ int mbok_read_device_errors(unsigned* flags);
  * that never landed would; the context stays usable.  No fault, no hang. */
 int mbok_check_wait_timeout(unsigned timeout_us, void* stream);
 
+/* Weight precision of the prefill GEMM (argument `precision` of mbok_gemm_ex). */
+#define MBOK_GEMM_AUTO 0      /* MBOK_GEMM_SPLIT when N <= MBOK_GEMM_SPLIT_MAX_N, else MBOK_GEMM_BF16 */
+#define MBOK_GEMM_BF16 1      /* each weight rounded once to bf16: one MMA per tile */
+#define MBOK_GEMM_SPLIT 2     /* each weight as two bf16 terms: two MMAs per tile */
+#define MBOK_GEMM_SPLIT_MAX_N 512
+
 /* Y[t][r] = sum_j Wt[r][j] * X[t][j] for t < T (prefill) on the tensor cores
- * (tcgen05, fp32 accumulation in tensor memory).  Wt is W in bf16: each fp16
- * scale is rounded to bf16 and the K signed scales of an element are summed
- * in bf16 while the tile is unpacked into shared memory.  Y is rounded to
- * bf16.  X: bf16 [T][N]; Y: bf16 [T][M]; both 16-byte aligned; 1 <= T <= 2^23.
- * Accuracy: the weight tile is W rounded through bf16 (each scale rounded
- * once, K - 1 bf16 additions), so each element of Wt is within about
- * (2K - 1) * 2^-8 * sum_k |alpha_k| of W; the scale rounding is the same for
- * a group's 128 columns.  For sign patterns that are not adversarial the
- * error of Y then stays within 1e-3 * sum_j |W x| + 2^-8 * |Y_exact| + 1e-6
- * per element with a margin that grows as sqrt(N): every output of the
- * tested N >= 4096 cases met it, while at N = 256, K = 2 about 7 in 10^5
- * outputs did not.  It is not a worst-case guarantee.  Waits inside the
- * kernel are bounded: see mbok_read_device_errors. */
+ * (tcgen05, fp32 accumulation in tensor memory).  K Boolean kernels give at
+ * most 2^K weight levels per (row, group) (Paper-Notes page, 关键设计); the
+ * kernel forms each level v = sum_k s_k alpha_k (s_k = +-1) in fp32 in kernel
+ * order -- exactly W[r][j] whenever a group's K scales lie within a factor
+ * 2^11 of one another -- and the tile Wt it multiplies is
+ *   MBOK_GEMM_BF16:  RN_bf16(v), one rounding: |Wt - W| <= 2^-8 |W|;
+ *   MBOK_GEMM_SPLIT: RN_bf16(v) + RN_bf16(v - RN_bf16(v)), two bf16 terms that
+ *                    both pass through the MMAs into the same accumulator:
+ *                    |Wt - W| <= 2^-16 |W|, at twice the tensor work.
+ * Y is rounded to bf16.  X: bf16 [T][N]; Y: bf16 [T][M]; both 16-byte
+ * aligned; 1 <= T <= 2^23.
+ * Accuracy: |Y - Y_exact| <= u * sum_j |W x| + (fp32 accumulation) + half a
+ * bf16 ulp of Y, with u = 2^-16 (split) or 2^-8 (bf16).  The split meets
+ * 1e-3 * sum_j |W x| + 2^-8 * |Y_exact| + 1e-6 for every output.  With one
+ * rounding the error of a group's weights shares the rounding of its few
+ * levels, so the bound above holds only on average: the tests hold every
+ * output to it for N >= 1024 (at N = 128 a few outputs in 10^5 miss), which
+ * is why MBOK_GEMM_AUTO splits for N <= 512.  Waits inside the kernel are
+ * bounded: see mbok_read_device_errors. */
+int mbok_gemm_ex(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+                 const uint16_t* X, int T, uint16_t* Y, int precision, void* stream);
+
+/* mbok_gemm_ex with MBOK_GEMM_AUTO. */
 int mbok_gemm(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
               const uint16_t* X, int T, uint16_t* Y, void* stream);
 

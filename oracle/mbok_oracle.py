@@ -416,6 +416,22 @@ def rel_l2(y, y_ref) -> float:
     return float(np.linalg.norm(y - y_ref)) / (den if den > 0 else 1.0)
 
 
+def round_bf16(v) -> np.ndarray:
+    """Round fp64 values once to bfloat16 (8 significant bits, the fp32
+    exponent range), nearest with ties to even; returned as fp64.
+
+    The prefill GEMM multiplies a bfloat16 weight tile: every weight W_rj,
+    exact in fp64 (reconstruct_rows), rounded once.  Written from the format's
+    definition: x = m * 2^e with 1/2 <= |m| < 1 (frexp), m scaled to 8 bits
+    and rounded half-to-even (numpy rint), the quantum fixed at 2^-133 below
+    the smallest normal 2^-126.  Finite inputs within the bf16 range only."""
+    x = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(x)
+    normal = np.rint(m * 256.0) * np.exp2(e.astype(np.float64) - 8.0)
+    sub = np.rint(x * 2.0 ** 133) * 2.0 ** -133
+    return np.where(np.abs(x) < 2.0 ** -126, sub, normal)
+
+
 def levels(K: int, alphas) -> set:
     """The set {sum_k s_k alpha_k : s in {-1,+1}^K} (at most 2^K weight levels)."""
     out = set()

@@ -11,3 +11,13 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+@pytest.fixture(autouse=True)
+def _output_guards(request):
+    """After every GPU test: the guard regions around its output buffers
+    (tests/helpers.py: guarded) must be intact."""
+    yield
+    if request.node.get_closest_marker("gpu") is not None:
+        import helpers
+        helpers.check_guards()

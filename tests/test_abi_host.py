@@ -101,8 +101,8 @@ def test_binding_refuses_cpu_tensors(L):
 
 def test_gemv_kernel_choice(L):
     import boolean_weight_matmul_b200 as mb
-    assert L.mbok_gemv_set_kernel(-1) == 1 and L.mbok_gemv_set_kernel(3) == 1
-    for k in (mb.GEMV_LOOKUP, mb.GEMV_TENSOR, mb.GEMV_AUTO):
+    assert L.mbok_gemv_set_kernel(-1) == 1 and L.mbok_gemv_set_kernel(5) == 1
+    for k in (mb.GEMV_LOOKUP, mb.GEMV_TENSOR, mb.GEMV_LOOKUP_SLABS, mb.GEMV_LOOKUP_ROWS, mb.GEMV_AUTO):
         assert L.mbok_gemv_set_kernel(k) == 0
     with mb.gemv_kernel(mb.GEMV_TENSOR):
         pass

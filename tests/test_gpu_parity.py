@@ -9,6 +9,7 @@ import pytest
 from oracle import mbok_oracle as O
 from boolean_weight_matmul_b200 import workloads as wl
 from helpers import (BF16_OUT_REL, GEMV_REL_L2, alpha_blocked_gpu, assert_close, ensure_built, gemm_gpu, x_dev,
+                     guarded, guarded_alpha, guarded_packed, check_guards,
                      gemv_gpu, packed_from_signs_gpu, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -54,9 +55,9 @@ def _residual_gpu(W: np.ndarray, K: int):
     import boolean_weight_matmul_b200 as mb
     M, N = W.shape
     Wd = to_dev(W)
-    packed = mb.empty_packed(K, M, N)
-    alpha = mb.empty_alpha(K, M, N)
-    R = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    packed = guarded_packed(K, M, N)
+    alpha = guarded_alpha(K, M, N)
+    R = guarded((M, N), torch.float32)
     mb.residual_binarize(Wd, M, N, K, 128, packed, alpha, R)
     torch.cuda.synchronize()
     return _words_u32(packed), alpha.cpu().numpy(), R.cpu().numpy()
@@ -159,8 +160,8 @@ def test_gemv_llama7b_mlp_residual_weights(which, K, batch):
     w = wl.mlp_7b(K, which, batch)
     M, N = w.M, w.N
     W = wl.w_normal(M, N, wl.seed_of(3, 1, 3))
-    packed = mb.empty_packed(K, M, N)
-    alpha = mb.empty_alpha(K, M, N)
+    packed = guarded_packed(K, M, N)
+    alpha = guarded_alpha(K, M, N)
     mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
     x = wl.x_normal(batch, N, wl.seed_of(3, 1, 2))
     y = gemv_gpu(packed, alpha, K, M, N, x, "bf16")
@@ -218,10 +219,12 @@ def test_gemv_deterministic():
 # The two GEMV kernels, each forced for every batch size
 # --------------------------------------------------------------------------
 
-KERNELS = {"lookup": 1, "tensor": 2}
+# lookup: the default lookup kernel (slabs); tensor: MMAs; lookup_rows: whole
+# rows with 4-bit tables where they fit (else slabs).
+KERNELS = {"lookup": 1, "tensor": 2, "lookup_rows": 4}
 
 
-@pytest.mark.parametrize("kernel", ["lookup", "tensor"])
+@pytest.mark.parametrize("kernel", ["lookup", "tensor", "lookup_rows"])
 @pytest.mark.parametrize("K", [1, 2, 3, 4])
 @pytest.mark.parametrize("M,N,batch", [(1, 128, 1), (7, 256, 3), (13, 640, 5), (129, 1024, 2),
                                        (64, 1536, 16), (24, 384, 6)])
@@ -270,7 +273,7 @@ def test_gemv_tensor_mlp_sampled(name, M, N, batch):
     assert_close(y, y_ref, E, GEMV_REL_L2, f"tensor {name} b{batch}")
 
 
-@pytest.mark.parametrize("kernel", ["lookup", "tensor"])
+@pytest.mark.parametrize("kernel", ["lookup", "tensor", "lookup_rows"])
 def test_gemv_kernel_flip_invariance_bitwise(kernel):
     # Negated signs (exact) times negated scales: the same y bit for bit.
     import boolean_weight_matmul_b200 as mb
@@ -288,8 +291,9 @@ def test_gemv_kernel_flip_invariance_bitwise(kernel):
             assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
 
 
+@pytest.mark.parametrize("kernel", ["lookup", "lookup_rows"])
 @pytest.mark.parametrize("M,N", [(4096, 4096), (300, 1536), (5120, 13824)])
-def test_gemv_static_weights_same_bits(M, N):
+def test_gemv_static_weights_same_bits(M, N, kernel):
     # Copying weights into shared memory before the dependency wait changes
     # no result: bit-identical outputs, also for a chain of launches whose
     # inputs the previous launch wrote.
@@ -300,7 +304,7 @@ def test_gemv_static_weights_same_bits(M, N):
     a = wl.alpha_decaying(K, M, N, 102)
     x = wl.x_normal(1, N, 103)
     p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
-    with mb.gemv_kernel(mb.GEMV_LOOKUP):
+    with mb.gemv_kernel(KERNELS[kernel]):
         mb.gemv_set_static_weights(False)
         y0 = gemv_gpu(p, al, K, M, N, x, "bf16")
         mb.gemv_set_static_weights(True)
@@ -312,7 +316,7 @@ def test_gemv_static_weights_same_bits(M, N):
             ys = []
             cur = xs
             for _ in range(3):
-                y = torch.empty(1, M, dtype=torch.float32, device="cuda")
+                y = guarded((1, M), torch.float32)
                 mb.gemv(p, al, K, M, N, 128, cur, mb.BF16, 1, y, ws)
                 ys.append(y)
                 if M == N:
@@ -353,9 +357,32 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
 
 
+@pytest.mark.parametrize("K,M,N", [
+    (3, 20000, 4096),    # 68 row pairs per CTA: more octets than ring slots, the ring wraps
+    (2, 40000, 512),     # more than 128 row pairs per CTA would be needed: a second wave of CTAs
+    (4, 1000, 10240),    # the widest rows the 4-bit tables cover (20 blocks of 512 columns)
+    (1, 333, 10368),     # one unit block more: the slab kernel takes over
+])
+def test_gemv_lookup_whole_rows_geometry(K, M, N):
+    # Row ranges that start and end inside octets, sampled around every CTA
+    # boundary of the whole-row lookup kernel plus random rows.
+    import boolean_weight_matmul_b200 as mb
+    pairs = (M + 1) // 2
+    ncta = min(148, pairs)
+    if -(-pairs // ncta) > 128:
+        ncta = -(-pairs // 128)
+    edges = np.array([2 * (c * pairs // ncta) for c in range(ncta)])
+    rows = np.unique(np.clip(np.concatenate([edges - 1, edges, edges + 1, [M - 1],
+                                             np.random.default_rng(M).choice(M, 200, replace=False)]), 0, M - 1))
+    with mb.gemv_kernel(mb.GEMV_LOOKUP_ROWS):
+        y, y_ref, E = _gemv_case(K, M, N, 1, "bf16", 8800 + M + N, "decaying", rows=rows)
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"whole-row lookup K={K} M={M} N={N}")
+    assert mb.read_device_errors() == 0
+
+
 def _multi_case(Ks, Ms, N, batch, x_dtype, seed):
     """mbok_gemv_multi over matrices with their own K and M, the separate
-    lookup-kernel calls, and the oracle (per matrix, concatenated)."""
+    slab lookup-kernel calls, and the oracle (per matrix, concatenated)."""
     import torch
     import boolean_weight_matmul_b200 as mb
     signs = [wl.random_signs(K, M, N, seed + 10 * i) for i, (K, M) in enumerate(zip(Ks, Ms))]
@@ -365,10 +392,10 @@ def _multi_case(Ks, Ms, N, batch, x_dtype, seed):
     alpha = [alpha_blocked_gpu(a, K, M, N) for a, K, M in zip(alphas, Ks, Ms)]
     xd = x_dev(x, x_dtype)
     dt = mb.F32 if x_dtype == "f32" else mb.BF16
-    y = torch.empty(batch, sum(Ms), dtype=torch.float32, device="cuda")
+    y = guarded((batch, sum(Ms)), torch.float32)
     mb.gemv_multi(packed, alpha, Ks, Ms, N, 128, xd, dt, batch, y, mb.zeros_multi_workspace(Ks, Ms, N))
     torch.cuda.synchronize()
-    with mb.gemv_kernel(mb.GEMV_LOOKUP):
+    with mb.gemv_kernel(mb.GEMV_LOOKUP_SLABS):
         sep = np.concatenate([gemv_gpu(p, a, K, M, N, x, x_dtype) for p, a, K, M in zip(packed, alpha, Ks, Ms)],
                              axis=1)
     refs = [O.linear(O.pack_signs(sg), a, K, M, N, x, x_dtype) for sg, a, K, M in zip(signs, alphas, Ks, Ms)]
@@ -386,7 +413,7 @@ def _multi_case(Ks, Ms, N, batch, x_dtype, seed):
 def test_gemv_multi_equals_separate_calls(Ks, Ms, N, batch, x_dtype):
     # Each row is computed as in its own matrix's launch (same tables, same
     # octet order, slabs added in order), so the fused outputs equal the
-    # separate lookup-kernel calls bit for bit, and the oracle within tolerance.
+    # separate slab lookup-kernel calls bit for bit, and the oracle within tolerance.
     y, sep, y_ref, E = _multi_case(Ks, Ms, N, batch, x_dtype, 12000 + N + sum(Ms))
     assert np.array_equal(y.view(np.uint32), sep.view(np.uint32))
     assert_close(y, y_ref, E, GEMV_REL_L2, f"multi K={Ks} M={Ms} N={N}")
@@ -434,7 +461,7 @@ def _svid_gpu(signs, s_in, s_out, x, x_dtype):
     si = to_dev(np.ascontiguousarray(s_in, dtype=np.float16).view(np.int16)).view(torch.float16)
     so = to_dev(np.ascontiguousarray(s_out, dtype=np.float16).view(np.int16)).view(torch.float16)
     xd = x_dev(x, x_dtype)
-    y = torch.empty(batch, M, dtype=torch.float32, device="cuda")
+    y = guarded((batch, M), torch.float32)
     ws = mb.zeros_svid_workspace(K, M, N, batch)
     mb.gemv_svid(packed, si, so, K, M, N, xd, mb.F32 if x_dtype == "f32" else mb.BF16, batch, y, ws)
     torch.cuda.synchronize()
@@ -489,7 +516,7 @@ def _refit_gpu(W, packed, K):
     import torch
     import boolean_weight_matmul_b200 as mb
     M, N = W.shape
-    out = mb.empty_alpha(K, M, N)
+    out = guarded_alpha(K, M, N)
     mb.refit_alpha(to_dev(W), packed, K, M, N, 128, out)
     torch.cuda.synchronize()
     return O.unblock_alpha(out.cpu().numpy(), K, M, N)
@@ -511,8 +538,8 @@ def test_refit_bit_exact_on_greedy_kernels_and_dependent_kernels():
     import boolean_weight_matmul_b200 as mb
     K, M, N = 3, 40, 768
     W = wl.w_normal(M, N, 9100)
-    packed = mb.empty_packed(K, M, N)
-    alpha = mb.empty_alpha(K, M, N)
+    packed = guarded_packed(K, M, N)
+    alpha = guarded_alpha(K, M, N)
     mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
     words = _words_u32(packed)
     signs = O.unpack_bits(words, K, M, N)
@@ -530,8 +557,8 @@ def test_refit_llama7b_gate_sampled():
     import boolean_weight_matmul_b200 as mb
     K, M, N = 3, 11008, 4096
     W = wl.w_normal(M, N, 9200)
-    packed = mb.empty_packed(K, M, N)
-    alpha = mb.empty_alpha(K, M, N)
+    packed = guarded_packed(K, M, N)
+    alpha = guarded_alpha(K, M, N)
     mb.residual_binarize(to_dev(W), M, N, K, 128, packed, alpha)
     got = _refit_gpu(W, packed, K)
     rows = np.sort(np.random.default_rng(3).choice(M, 64, replace=False))
@@ -548,10 +575,10 @@ def _svid_binarize_gpu(W, K, iters=6):
     import torch
     import boolean_weight_matmul_b200 as mb
     M, N = W.shape
-    packed = mb.empty_packed(K, M, N)
-    s_in = torch.empty(K, N, dtype=torch.float16, device="cuda")
-    s_out = torch.empty(K, M, dtype=torch.float16, device="cuda")
-    R = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    packed = guarded_packed(K, M, N)
+    s_in = guarded((K, N), torch.float16)
+    s_out = guarded((K, M), torch.float16)
+    R = guarded((M, N), torch.float32)
     mb.svid_binarize(to_dev(W), M, N, K, iters, packed, s_in, s_out, R)
     torch.cuda.synchronize()
     return _words_u32(packed), s_in.cpu().numpy(), s_out.cpu().numpy(), R.cpu().numpy()
@@ -603,7 +630,7 @@ def test_svid_binarize_then_gemv_matches_oracle():
     packed = to_dev(words.view(np.int32))
     si = to_dev(s_in.view(np.int16)).view(torch.float16)
     so = to_dev(s_out.view(np.int16)).view(torch.float16)
-    yd = torch.empty(1, M, dtype=torch.float32, device="cuda")
+    yd = guarded((1, M), torch.float32)
     mb.gemv_svid(packed, si, so, K, M, N, x_dev(x, "bf16"), mb.BF16, 1, yd, mb.zeros_svid_workspace(K, M, N))
     torch.cuda.synchronize()
     y_ref, E = O.linear_svid(words, s_in, s_out, K, M, N, x, "bf16")
@@ -637,6 +664,61 @@ def test_gemm_small(K, M, N, T):
     assert_close(Y, Y_ref, E, None, f"gemm K={K} M={M} N={N} T={T}", out_rel=BF16_OUT_REL)
 
 
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+def test_gemm_weight_tile_is_each_level_rounded_once(K, split):
+    # With X the identity (token t = unit vector e_t) every output is one
+    # weight of the tile: Y[t][r] = Wt[r][t] (one nonzero product per tile
+    # term, fp32 accumulation).  With one rounding it must be the exact weight
+    # W[r][t] = sum_k alpha_k b_k rounded once to bf16, bit for bit; with the
+    # split, RN_bf16(hi + lo) where hi = RN_bf16(W) and lo = RN_bf16(W - hi),
+    # i.e. again RN_bf16(W) after the output's rounding.  Rows and columns span
+    # two row tiles, two groups and every column of a stage.
+    import boolean_weight_matmul_b200 as mb
+    M, N = 256, 256
+    s = wl.random_signs(K, M, N, 870 + K)
+    a = wl.alpha_decaying(K, M, N, 875 + K)
+    eye = np.zeros((N, N), dtype=np.float32)
+    np.fill_diagonal(eye, 1.0)
+    X = (eye.view(np.uint32) >> 16).astype(np.uint16)   # bf16 bit patterns of 0 and 1
+    Y = gemm_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, X,
+                 precision=mb.GEMM_SPLIT if split else mb.GEMM_BF16)
+    W = O.reconstruct_W(O.pack_signs(s), a, K, M, N)
+    want = O.round_bf16(W).T
+    bad = np.argwhere(Y != want)
+    assert bad.size == 0, (f"{len(bad)} weights differ from RN_bf16(W), e.g. token {bad[0][0]} row {bad[0][1]}: "
+                           f"got {Y[tuple(bad[0])]} want {want[tuple(bad[0])]}")
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+@pytest.mark.parametrize("N", [128, 256, 512, 1024])
+def test_gemm_small_n_every_output(K, N):
+    # Small N is where the accumulation bound 1e-3 * sum|W x| is tightest
+    # against the weight tile's rounding: 4096 tokens, every output checked,
+    # with mbok_gemm's own choice (the split up to N = 512, one rounding above).
+    M, T = 256, 4096
+    s = wl.random_signs(K, M, N, 850 + 10 * K + N)
+    a = wl.alpha_decaying(K, M, N, 851 + 10 * K + N)
+    X = wl.x_normal(T, N, 852 + 10 * K + N)
+    Y = gemm_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, X)
+    Y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, X, "bf16")
+    assert_close(Y, Y_ref, E, None, f"gemm K={K} N={N} T={T}", out_rel=BF16_OUT_REL)
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_gemm_split_at_prefill_width(K):
+    # The split asked for explicitly at N = 4096: same bound, sampled rows.
+    import boolean_weight_matmul_b200 as mb
+    M, N, T = 512, 4096, 1024
+    s = wl.random_signs(K, M, N, 860 + K)
+    a = wl.alpha_decaying(K, M, N, 861 + K)
+    X = wl.x_normal(T, N, 862 + K)
+    Y = gemm_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, X, precision=mb.GEMM_SPLIT)
+    rows = np.sort(np.random.default_rng(863).choice(M, 64, replace=False))
+    Y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, X, "bf16", rows=rows)
+    assert_close(Y[:, rows], Y_ref, E, None, f"gemm split K={K}", out_rel=BF16_OUT_REL)
+
+
 def test_gemm_prefill_q_proj_sampled():
     # LLaMA-7B q_proj prefill: K=3, 4096 x 4096, 2048 tokens; 128 sampled rows.
     w = wl.PREFILL_7B
@@ -654,10 +736,7 @@ def test_gemm_several_tiles_per_cta():
     # More tiles than SMs (4096 rows = 16 row tiles x 18 token tiles of 4096
     # tokens): persistent CTAs take a second tile and reuse their tensor-memory
     # accumulators after the epilogue drains them.  Sampled rows from every
-    # row tile, every token.  N = 4096 as in the prefill configuration: the
-    # bf16 weight tile meets the per-element bound with a margin that grows as
-    # sqrt(N), and at N = 256 a few outputs in 10^5 miss it (documented in the
-    # header), which is not what this test is about.
+    # row tile, every token.
     import boolean_weight_matmul_b200 as mb
     K, M, N, T = 3, 4096, 4096, 4096
     s = wl.random_signs(K, M, N, 881)
@@ -680,3 +759,16 @@ def test_gemm_no_wait_gave_up():
     Y_ref, E = O.linear(O.pack_signs(s), a, 2, 256, 512, X, "bf16")
     assert_close(Y, Y_ref, E, None, "gemm after-run check", out_rel=BF16_OUT_REL)
     assert mb.read_device_errors() == 0
+
+
+def test_output_guards_catch_a_write_past_the_end():
+    # The guard check itself: a byte written just past an output (here by the
+    # host, through torch) must be reported.
+    import torch
+    y = guarded((3, 5), torch.float32)
+    y.fill_(1.0)
+    base = y.view(-1).view(torch.uint8)
+    raw = torch.as_strided(base, (base.numel() + 1,), (1,))   # one byte beyond the end
+    raw[-1] = 0
+    with pytest.raises(AssertionError):
+        check_guards()

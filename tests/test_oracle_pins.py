@@ -491,3 +491,28 @@ def test_svid_residual_shrinks_and_signs_of_zero():
         _, R = O.svid_step(R, so, si)
         norms.append(np.linalg.norm(R.astype(np.float64)))
     assert all(a > b for a, b in zip(norms, norms[1:]))
+
+
+def test_round_bf16_pins():
+    """The bf16 rounding used for the GEMM's weight tile, pinned without
+    restating it: representable values are fixed points, midpoints go to the
+    even neighbour, fp64 inputs just past a midpoint round up (a detour
+    through fp32 would round them down), and on fp32 inputs it agrees with
+    torch's float32 -> bfloat16 conversion."""
+    import torch
+    # representable: 8 significant bits
+    rep = np.array([1.0, -1.0, 1.0 + 2.0 ** -7, 3.0, 0.0, 2.0 ** -126, -(2.0 ** 100), 1.9921875])
+    assert np.array_equal(O.round_bf16(rep), rep)
+    # ties to even: spacing at 1.0 is 2^-7
+    assert O.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert O.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.round_bf16(-(1.0 + 2.0 ** -8)) == -1.0
+    # single rounding from fp64: just above the midpoint rounds up
+    assert O.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -40) == 1.0 + 2.0 ** -7
+    assert np.float32(1.0 + 2.0 ** -8 + 2.0 ** -40) == np.float32(1.0 + 2.0 ** -8)
+    # agreement with a library conversion on fp32 values (normal and subnormal)
+    rng = np.random.default_rng(7)
+    v = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+                        rng.standard_normal(2000) * 2.0 ** -130]).astype(np.float32)
+    lib = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_bf16(v.astype(np.float64)), lib)
