@@ -352,6 +352,22 @@ def run_gpu(a):
 
     # Eagerly: one Python call per layer (host launch overhead included).
     eager_ms = time_e2e(e2e_step)
+    # Eagerly through the C ABI itself: ctypes calls of mbok_gemv with raw
+    # pointers prepared once (the binding's checks bypassed), the same copies.
+    lib_gemv = mb.lib().mbok_gemv
+    sp = stream.cuda_stream
+    wsp, wsn = ws.data_ptr(), ws.numel()
+    args = [(packed[l].data_ptr(), alphas[l].data_ptr(), x_dev[l].data_ptr(), y_dev[l].data_ptr())
+            for l in range(L)]
+
+    def e2e_abi_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        for (pp, pa, px, py) in args:
+            lib_gemv(pp, pa, K, M, N, 128, px, mb.BF16, 1, py, wsp, wsn, sp)
+        y_host.copy_(y_dev, non_blocking=True)
+    with torch.cuda.stream(stream):
+        assert lib_gemv(args[0][0], args[0][1], K, M, N, 128, args[0][2], mb.BF16, 1, args[0][3], wsp, wsn, sp) == 0
+    abi_ms = time_e2e(e2e_abi_step)
     # As a serving loop runs it: the whole step (copies and calls) captured
     # once in a CUDA graph and replayed; the copies still run every step.
     with torch.cuda.stream(stream):
@@ -367,7 +383,11 @@ def run_gpu(a):
            "path": "mbok_gemv via the C ABI, pinned host x/y copied in and out every step; the step "
                    "(copies + calls) captured once in a CUDA graph and replayed",
            "eager": {"value": replica_rate(L * bytes_per_layer, eager_ms, world) / 1e9, "ms_per_step": eager_ms,
-                     "path": "the same step issued eagerly from Python, one call per layer"}}
+                     "path": "the same step issued eagerly from Python, one binding call per layer"},
+           "abi_direct": {"value": replica_rate(L * bytes_per_layer, abi_ms, world) / 1e9, "ms_per_step": abi_ms,
+                          "us_per_call": 1e3 * abi_ms / L,
+                          "path": "the same step issued eagerly as direct ctypes calls of mbok_gemv (C ABI, "
+                                  "pointers prepared once), copies included"}}
     del e2e_graph
 
     del graph
@@ -384,6 +404,14 @@ def run_gpu(a):
         dist.destroy_process_group()
     if rank != 0:
         return
+    # Secondary rows: one short JSON line each, printed before the headline
+    # (which stays the last line); the headline carries a compact summary.
+    compact = None
+    if extras:
+        compact = {}
+        for name, row in extras.items():
+            print(json.dumps({"row": name, **row}), flush=True)
+            compact[name] = row_summary(row)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -404,9 +432,17 @@ def run_gpu(a):
         "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": a.steps * L * launches_per_gemv,
-        "rows": extras,
+        "rows": compact,
     }
     print(json.dumps(line), flush=True)
+
+
+def row_summary(row: dict) -> list:
+    """[time, rate, fraction of peak] of a secondary row, for the headline."""
+    t = row.get("us", row.get("us_per_layer", row.get("ms_per_token", row.get("ms"))))
+    rate = row.get("tflops", row.get("tokens_per_s", row.get("gbs", row.get("gbs_of_w", row.get("gbs_in")))))
+    frac = row.get("frac_of_bf16_peak", row.get("frac_of_hbm"))
+    return [None if v is None else round(float(v), 4) for v in (t, rate, frac)]
 
 
 def run_extras(torch, mb, wl, dev, peaks, a):
@@ -439,13 +475,16 @@ def run_gemm_row(torch, mb, wl, dev, peaks, stream, g, out):
                   K, M, N, alpha)
     X = torch.randn(T, N, device=dev, generator=g).to(torch.bfloat16)
     Y = torch.empty(T, M, dtype=torch.bfloat16, device=dev)
-    ms, gr = time_graph(torch, lambda: mb.gemm(packed, alpha, K, M, N, 128, X, T, Y, stream=stream),
-                        10, 3, stream)
-    tflops = 2.0 * M * N * T / (ms * 1e-3) / 1e12
-    out["prefill_gemm_llama7b_q_proj_k3_t2048"] = {
-        "us": 1e3 * ms, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-        "peak_tflops": peaks["bf16_tflops"], "kernel": "gemm_tc_kernel<3>"}
-    del gr, packed, X, Y
+    for (suffix, prec, kern) in (("", mb.GEMM_AUTO, "gemm_tc_kernel<3,false> (one bf16 rounding per weight)"),
+                                 ("_split", mb.GEMM_SPLIT, "gemm_tc_kernel<3,true> (hi + lo bf16 terms)")):
+        ms, gr = time_graph(torch, lambda: mb.gemm(packed, alpha, K, M, N, 128, X, T, Y, stream=stream,
+                                                   precision=prec), 10, 3, stream)
+        tflops = 2.0 * M * N * T / (ms * 1e-3) / 1e12
+        out["prefill_gemm_llama7b_q_proj_k3_t2048" + suffix] = {
+            "us": 1e3 * ms, "tflops": tflops, "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "peak_tflops": peaks["bf16_tflops"], "kernel": kern}
+        del gr
+    del packed, X, Y
     torch.cuda.empty_cache()
 
 
@@ -455,6 +494,7 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
     # weight copies per graph that they exceed L2 (>= 150 MB).
     shapes = (("q_proj", 3, 4096, 4096), ("gate", 3, 11008, 4096), ("down", 2, 4096, 11008))
     kernels = (("lookup", mb.GEMV_LOOKUP, True), ("lookup_weights_after_wait", mb.GEMV_LOOKUP, False),
+               ("lookup_rows", mb.GEMV_LOOKUP_ROWS, True),
                ("tensor", mb.GEMV_TENSOR, True))
     for (name, K, M, N) in shapes:
         bpl = mb.packed_bytes(K, M, N) + 2 * mb.alpha_elems(K, M, N)
@@ -472,7 +512,8 @@ def run_small_batch_rows(torch, mb, wl, dev, peaks, stream, g, out):
             x = torch.randn(batch, N, device=dev, generator=g).to(torch.bfloat16)
             y = torch.empty(batch, M, dtype=torch.float32, device=dev)
             for (kname, kcode, static) in kernels:
-                if batch > 1 and (kname.endswith("after_wait") or (name == "q_proj" and kname == "lookup")):
+                if batch > 1 and (kname.endswith("after_wait") or kname == "lookup_rows"
+                                  or (name == "q_proj" and kname == "lookup")):
                     continue
 
                 def fn():
