@@ -51,8 +51,12 @@ def args_parse():
                    help="comma-separated secondary rows to run")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile-gemv", default=None, metavar="K,M,N,BATCH,KERNEL",
-                   help="profiling helper: run four launches of one GEMV (KERNEL 0 auto, 1 lookup, "
-                        "2 tensor) with L2 flushed between them, print nothing else, and exit")
+                   help="profiling helper: run four launches of one GEMV (KERNEL as mbok_gemv_set_kernel: "
+                        "0 auto, 1 lookup, 2 tensor, 3 slab lookup, 4 whole-row lookup) with L2 flushed "
+                        "between them, print nothing else, and exit")
+    p.add_argument("--profile-gemm", default=None, metavar="K,M,N,T,PRECISION",
+                   help="profiling helper: run three launches of one prefill GEMM (PRECISION as "
+                        "mbok_gemm_ex: 0 auto, 1 bf16, 2 split), print nothing else, and exit")
     return p.parse_args()
 
 
@@ -65,21 +69,25 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash(name: str) -> str:
-    with open(os.path.join(ROOT, "boolean_weight_matmul_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_source_hash(names) -> str:
+    """sha256 (16 hex digits) of the listed csrc files, concatenated in order."""
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "boolean_weight_matmul_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_file: str, key: str):
-    """Per-launch DRAM bytes from the committed ncu summary, or None when the
-    kernel source changed since the counters were taken."""
+def ncu_traffic(key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, or None when any
+    source file of the kernel changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(key)
-    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+    if not e or e.get("source_sha256_16") != kernel_source_hash(e.get("sources", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -320,7 +328,7 @@ def run_gpu(a):
     launches_per_gemv = 2 if N > 512 else 1
     us_per_layer = 1e3 * ms / L
     achieved = bytes_per_layer / (us_per_layer * 1e-6) / 1e9
-    traffic = ncu_traffic("gemv_lut.cu", "gemv_lut8_q_proj_k3_4096x4096")
+    traffic = ncu_traffic("gemv_lut8_q_proj_k3_4096x4096")
 
     # End to end through the C ABI with host buffers: per step, copy the L
     # activation vectors host->device, run the L GEMVs, copy the L outputs back.
@@ -714,10 +722,33 @@ def profile_gemv(spec: str):
     torch.cuda.synchronize()
 
 
+def profile_gemm(spec: str):
+    """Three launches of one prefill GEMM on random weights (for an ncu capture)."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    mbuild.build()
+    K, M, N, T, prec = (int(v) for v in spec.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                           device=dev, generator=g)
+    alpha = (torch.rand(mb.alpha_elems(K, M, N), device=dev, generator=g) * 0.01 + 0.005).to(torch.float16)
+    X = torch.randn(T, N, device=dev, generator=g).to(torch.bfloat16)
+    Y = torch.empty(T, M, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        mb.gemm(packed, alpha, K, M, N, 128, X, T, Y, precision=prec)
+    torch.cuda.synchronize()
+
+
 def main():
     a = args_parse()
     if a.profile_gemv:
         profile_gemv(a.profile_gemv)
+        return
+    if a.profile_gemm:
+        profile_gemm(a.profile_gemm)
         return
     if a.impl == "reference":
         run_reference(a)
