@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "mbok_gemv": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp], i),
             "mbok_gemm": ([vp, vp, i, i, i, i, vp, i, vp, vp], i),
             "mbok_gemm_ex": ([vp, vp, i, i, i, i, vp, i, vp, i, vp], i),
+            "mbok_gemv_ex": ([vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, i, i, vp], i),
             "mbok_gemv_noalloc": ([vp, vp, i, i, i, i, vp, i, i, vp, vp], i),
             "mbok_read_device_errors": ([ctypes.POINTER(ctypes.c_uint)], i),
             "mbok_check_wait_timeout": ([ctypes.c_uint, vp], i),
@@ -195,12 +196,21 @@ def refit_alpha(W, packed, K, M, N, group, alpha_out, stream=None) -> None:
     _check(lib().mbok_refit_alpha(pw, pp, K, M, N, group, po, _stream(stream)), "mbok_refit_alpha")
 
 
-def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=None) -> None:
+def gemv(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, stream=None, kernel=None,
+         weights_static=None) -> None:
+    """mbok_gemv; mbok_gemv_ex when a kernel choice or a static-weights flag
+    is given (the other then takes its default: GEMV_AUTO, static)."""
     ws_bytes = 0 if workspace is None else (workspace.numel() * workspace.element_size()
                                             if isinstance(workspace, torch.Tensor) else 0)
     pp, pa, px, py, pws = _ptrs(packed, alpha, x, y, workspace)
-    _check(lib().mbok_gemv(pp, pa, K, M, N, group, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
-           "mbok_gemv")
+    if kernel is None and weights_static is None:
+        _check(lib().mbok_gemv(pp, pa, K, M, N, group, px, x_dtype, batch, py, pws, ws_bytes, _stream(stream)),
+               "mbok_gemv")
+    else:
+        k = GEMV_AUTO if kernel is None else int(kernel)
+        ws_flag = 1 if weights_static is None or weights_static else 0
+        _check(lib().mbok_gemv_ex(pp, pa, K, M, N, group, px, x_dtype, batch, py, pws, ws_bytes, k, ws_flag,
+                                  _stream(stream)), "mbok_gemv_ex")
 
 
 def _int_array(vals):

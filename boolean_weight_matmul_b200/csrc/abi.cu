@@ -46,21 +46,21 @@ std::atomic<int> gemv_kernel_choice{MBOK_GEMV_AUTO};
 // (see mbok_gemv_set_static_weights).
 std::atomic<bool> gemv_weights_static{true};
 
-// One decode GEMV call: a lookup-table kernel once per vector -- 512-column
-// slabs with 8-bit tables and a combine launch, or, when asked for, whole rows
-// with 4-bit tables in one launch where they fit one CTA (N <= 10240) -- or
-// the tensor-core kernel over the whole batch.
+// One decode GEMV call with kernel choice `choice` (MBOK_GEMV_*): a
+// lookup-table kernel once per vector -- 512-column slabs with 8-bit tables
+// and a combine launch, or, when asked for, whole rows with 4-bit tables in
+// one launch where they fit one CTA (N <= 10240) -- or the tensor-core kernel
+// over the whole batch.  The slab kernel is the default lookup kernel: on B200
+// it measured faster at the LLaMA shapes (the whole-row kernel saves the
+// combine launch but does twice the lookups).
 cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
-                        bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
+                        bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream, int choice,
+                        bool weights_static) {
   bool tensor = batch > 1;
-  const int choice = gemv_kernel_choice.load(std::memory_order_relaxed);
   if (choice == MBOK_GEMV_LOOKUP || choice == MBOK_GEMV_LOOKUP_SLABS || choice == MBOK_GEMV_LOOKUP_ROWS)
     tensor = false;
   if (choice == MBOK_GEMV_TENSOR) tensor = true;
-  const bool weights_static = gemv_weights_static.load(std::memory_order_relaxed);
   if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream);
-  // Whole rows only when asked for: on B200 the slab kernel is measured
-  // faster on the LLaMA shapes (see the design notes).
   const bool rows = choice == MBOK_GEMV_LOOKUP_ROWS && gemv_lut4_supported(s);
   const size_t xbytes = x_f32 ? 4 : 2;
   for (int b = 0; b < batch; ++b) {
@@ -71,6 +71,15 @@ cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shap
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// The same with the process-wide choices (mbok_gemv_set_kernel,
+// mbok_gemv_set_static_weights), read once.
+cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shape& s, const void* x,
+                        bool x_f32, int batch, float* y, void* workspace, cudaStream_t stream) {
+  return launch_gemv(packed, alpha, s, x, x_f32, batch, y, workspace, stream,
+                     gemv_kernel_choice.load(std::memory_order_relaxed),
+                     gemv_weights_static.load(std::memory_order_relaxed));
 }
 }  // namespace mbok
 
@@ -198,9 +207,9 @@ int mbok_refit_alpha(const float* W, const uint32_t* packed, int K, int M, int N
                                       reinterpret_cast<__half*>(alpha), as_stream(stream)));
 }
 
-int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
-              const void* x, int x_dtype, int batch, float* y, void* workspace,
-              size_t workspace_bytes, void* stream) {
+int mbok_gemv_ex(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+                 const void* x, int x_dtype, int batch, float* y, void* workspace, size_t workspace_bytes,
+                 int kernel, int weights_static, void* stream) {
   const int st = check_shape(K, M, N);
   if (st != MBOK_OK) return st;
   if (group != MBOK_GROUP) return MBOK_ERR_UNSUPPORTED;
@@ -208,6 +217,8 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
     return MBOK_ERR_INVALID_ARG;
   if (x_dtype != MBOK_F32 && x_dtype != MBOK_BF16) return MBOK_ERR_INVALID_ARG;
   if (batch < 1 || batch > MBOK_MAX_BATCH) return MBOK_ERR_INVALID_ARG;
+  if (kernel < MBOK_GEMV_AUTO || kernel > MBOK_GEMV_LOOKUP_ROWS) return MBOK_ERR_INVALID_ARG;
+  if (weights_static != 0 && weights_static != 1) return MBOK_ERR_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(alpha, 16) || !aligned(x, 16) || !aligned(y, 4))
     return MBOK_ERR_ALIGN;
   const Shape s = make_shape(K, M, N);
@@ -215,7 +226,15 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 16)))
     return MBOK_ERR_WORKSPACE;
   return from_cuda(launch_gemv(reinterpret_cast<const uint8_t*>(packed), alpha, s, x, x_dtype == MBOK_F32,
-                               batch, y, workspace, as_stream(stream)));
+                               batch, y, workspace, as_stream(stream), kernel, weights_static == 1));
+}
+
+int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+              const void* x, int x_dtype, int batch, float* y, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  return mbok_gemv_ex(packed, alpha, K, M, N, group, x, x_dtype, batch, y, workspace, workspace_bytes,
+                      gemv_kernel_choice.load(std::memory_order_relaxed),
+                      gemv_weights_static.load(std::memory_order_relaxed) ? 1 : 0, stream);
 }
 
 // Argument checks of the multi-matrix GEMV's shape arrays; MBOK_OK or the

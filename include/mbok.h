@@ -203,6 +203,18 @@ int mbok_gemv(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N
               const void* x, int x_dtype, int batch, float* y, void* workspace,
               size_t workspace_bytes, void* stream);
 
+/* mbok_gemv with the two process-wide choices given per call instead:
+ *   kernel         : MBOK_GEMV_AUTO, _LOOKUP, _TENSOR, _LOOKUP_SLABS or
+ *                    _LOOKUP_ROWS, as for mbok_gemv_set_kernel;
+ *   weights_static : 1 or 0, as for mbok_gemv_set_static_weights.
+ * Other arguments, results and accuracy as mbok_gemv; mbok_gemv is this call
+ * with the process-wide values.  Nothing process-wide is read or written, so
+ * host threads may issue calls with different choices concurrently.
+ * MBOK_ERR_INVALID_ARG for any other kernel or weights_static value. */
+int mbok_gemv_ex(const uint32_t* packed, const uint16_t* alpha, int K, int M, int N, int group,
+                 const void* x, int x_dtype, int batch, float* y, void* workspace, size_t workspace_bytes,
+                 int kernel, int weights_static, void* stream);
+
 /* Bytes of device workspace mbok_gemv_svid needs (same rules as
  * mbok_gemv_workspace_bytes; one workspace may serve both calls if it has
  * the larger of the two sizes). */

@@ -218,3 +218,14 @@ def test_gemv_multi_sizes_and_argument_errors(L):
     assert call(2, [1, 2], [8, 8], batch=17) == 1       # batch out of range
     assert call(2, [1, 2], [8, 8], x=0x3008) == 3       # x not 16-byte aligned
     assert call(2, [1, 2], [8, 8]) == 6                 # N > 512 needs a workspace
+
+
+def test_gemv_ex_argument_checks(L):
+    # Per-call kernel choice and static-weights flag: invalid values are
+    # refused on the host before anything is launched (the pointers are never
+    # dereferenced).
+    P = 1 << 20
+    assert L.mbok_gemv_ex(P, P, 3, 64, 512, 128, P, 1, 1, P, P, 1 << 20, 5, 1, None) == 1
+    assert L.mbok_gemv_ex(P, P, 3, 64, 512, 128, P, 1, 1, P, P, 1 << 20, -1, 1, None) == 1
+    assert L.mbok_gemv_ex(P, P, 3, 64, 512, 128, P, 1, 1, P, P, 1 << 20, 1, 2, None) == 1
+    assert L.mbok_gemv_ex(P, P, 3, 64, 500, 128, P, 1, 1, P, P, 1 << 20, 1, 1, None) == 2

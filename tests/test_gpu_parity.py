@@ -357,6 +357,32 @@ def test_gemv_tensor_deterministic_and_batch_independent():
     assert np.array_equal(y8[5].view(np.uint32), y_one[0].view(np.uint32))
 
 
+@pytest.mark.parametrize("kernel", ["lookup", "tensor", "lookup_rows"])
+def test_gemv_ex_per_call_choice_equals_process_wide(kernel):
+    # mbok_gemv_ex with a kernel and static-weights flag per call gives, bit for
+    # bit, what mbok_gemv gives under the same process-wide choices.
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    K, M, N, batch = 3, 264, 1536, 3
+    s = wl.random_signs(K, M, N, 71)
+    a = wl.alpha_decaying(K, M, N, 72)
+    x = x_dev(wl.x_normal(batch, N, 73), "bf16")
+    p, al = packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N)
+    ws = mb.zeros_workspace(K, M, N, batch)
+    for static in (True, False):
+        y0 = guarded((batch, M), torch.float32)
+        with mb.gemv_kernel(KERNELS[kernel]):
+            mb.gemv_set_static_weights(static)
+            try:
+                mb.gemv(p, al, K, M, N, 128, x, mb.BF16, batch, y0, ws)
+            finally:
+                mb.gemv_set_static_weights(True)
+        y1 = guarded((batch, M), torch.float32)
+        mb.gemv(p, al, K, M, N, 128, x, mb.BF16, batch, y1, ws, kernel=KERNELS[kernel], weights_static=static)
+        torch.cuda.synchronize()
+        assert torch.equal(y0.view(torch.int32), y1.view(torch.int32))
+
+
 @pytest.mark.parametrize("K,M,N", [
     (3, 20000, 4096),    # 68 row pairs per CTA: more octets than ring slots, the ring wraps
     (2, 40000, 512),     # more than 128 row pairs per CTA would be needed: a second wave of CTAs
