@@ -27,7 +27,7 @@ cudaError_t launch_gemv_svid(const uint8_t*, const uint16_t*, const uint16_t*, c
 unsigned gemv_mma_error_flags();
 cudaError_t launch_wait_timeout_probe(unsigned, cudaStream_t);
 cudaError_t launch_gemv_mma(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int,
-                            float*, cudaStream_t);
+                            float*, cudaStream_t, bool);
 cudaError_t launch_gemv(const uint8_t*, const uint16_t*, const Shape&, const void*, bool, int, float*,
                         void*, cudaStream_t);
 
@@ -60,7 +60,7 @@ cudaError_t launch_gemv(const uint8_t* packed, const uint16_t* alpha, const Shap
   if (choice == MBOK_GEMV_LOOKUP || choice == MBOK_GEMV_LOOKUP_SLABS || choice == MBOK_GEMV_LOOKUP_ROWS)
     tensor = false;
   if (choice == MBOK_GEMV_TENSOR) tensor = true;
-  if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream);
+  if (tensor) return launch_gemv_mma(packed, alpha, s, x, x_f32, batch, y, stream, weights_static);
   const bool rows = choice == MBOK_GEMV_LOOKUP_ROWS && gemv_lut4_supported(s);
   const size_t xbytes = x_f32 ? 4 : 2;
   for (int b = 0; b < batch; ++b) {

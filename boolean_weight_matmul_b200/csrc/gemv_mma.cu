@@ -34,7 +34,9 @@
 //    16(4c+t) + 4j .. +3).  B uses the same permutation, which is simply 16
 //    consecutive activations of that unit per thread.
 //  * Launches use programmatic dependent launch: before waiting on the
-//    previous grid a CTA only asks L2 to prefetch its tile's bits and scales.
+//    previous grid a CTA asks L2 to prefetch its tile's bits and scales and,
+//    unless told that an earlier kernel on the stream may write the weights,
+//    issues the copies of its first slices.
 //  * Every mbarrier wait is bounded (1 s); on timeout the CTA records an
 //    error flag (bit 2 of mbok_read_device_errors), skips the rest of its
 //    work, waits (bounded) for its copies in flight and exits without
@@ -77,6 +79,7 @@ struct GemvMmaParams {
   float* y;             // [nb][M]
   Shape s;
   int nb;               // vectors in this launch
+  int weights_static;   // bits and scales may be read before the grid dependency wait
   uint32_t mul[8];      // 2^(15 - 2i): sign_pair factors
 };
 
@@ -474,6 +477,12 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
     }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    // Weights that no earlier kernel on the stream writes: the ring's first
+    // slices are copied before the dependency wait.
+    if (p.weights_static) {
+      for (; c.issued < kMmaStages && c.issued < c.n_slices; ++c.issued)
+        issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, smem + c.issued * stage_bytes, &full[c.issued]);
+    }
   }
   // Before the dependency wait: L2 prefetch of this tile's bits and scales.
   if (c.warp == 1) {
@@ -643,7 +652,8 @@ unsigned gemv_mma_error_flags() {
 // Y[b] = W X[b] for b < batch (x: [batch][N], y: [batch][M]); launches cover
 // up to 16 bf16 or 5 fp32 vectors each.
 cudaError_t launch_gemv_mma(const uint8_t* packed, const uint16_t* alpha, const Shape& s,
-                            const void* x, bool x_f32, int batch, float* y, cudaStream_t stream) {
+                            const void* x, bool x_f32, int batch, float* y, cudaStream_t stream,
+                            bool weights_static) {
   const int per_launch = x_f32 ? (8 * kMaxNT) / 3 : 8 * kMaxNT;
   const size_t x_elem = x_f32 ? 4 : 2;
   for (int b0 = 0; b0 < batch; b0 += per_launch) {
@@ -654,6 +664,7 @@ cudaError_t launch_gemv_mma(const uint8_t* packed, const uint16_t* alpha, const 
     p.y = y + size_t(b0) * s.M;
     p.s = s;
     p.nb = batch - b0 < per_launch ? batch - b0 : per_launch;
+    p.weights_static = weights_static ? 1 : 0;
     for (int i = 0; i < 8; ++i) p.mul[i] = 1u << (15 - 2 * i);
     cudaError_t e;
     switch (s.K) {
