@@ -54,6 +54,8 @@ def args_parse():
                    help="profiling helper: run four launches of one GEMV (KERNEL as mbok_gemv_set_kernel: "
                         "0 auto, 1 lookup, 2 tensor, 3 slab lookup, 4 whole-row lookup) with L2 flushed "
                         "between them, print nothing else, and exit")
+    p.add_argument("--phase-profile", default=None, metavar="K,M,N,LAYERS",
+                   help="per-phase split of the decode GEMV chain (profiling build with phase stamps)")
     p.add_argument("--profile-gemm", default=None, metavar="K,M,N,T,PRECISION",
                    help="profiling helper: run three launches of one prefill GEMM (PRECISION as "
                         "mbok_gemm_ex: 0 auto, 1 bf16, 2 split), print nothing else, and exit")
@@ -742,8 +744,112 @@ def profile_gemm(spec: str):
     torch.cuda.synchronize()
 
 
+def phase_profile(spec: str):
+    """Per-phase split of a chain of batch-1 decode GEMVs (slab lookup kernel +
+    slab combine), from the profiling build's per-CTA globaltimer stamps.  The
+    chain of LAYERS distinct weight copies is captured in a CUDA graph (as in
+    the headline) and replayed; the stamps of the last replay are read back.
+    Per layer l, on the critical path:
+      handoff_in  = first main CTA past its dependency wait - last combine CTA of layer l-1 done
+      x_tables    = last main CTA with its tables built - first main CTA past the wait
+      loop        = last warp out of the streaming loop - last CTA with tables built
+      drain       = last warp's copies drained - last warp out of the loop
+      handoff_mid = first combine CTA past its wait - main kernel done
+      combine     = last combine CTA done - first combine CTA past its wait
+    (the six terms add up to the layer's period)."""
+    import ctypes
+    import statistics
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    from boolean_weight_matmul_b200 import workloads as wl
+    mbuild.build()
+    path = mbuild.build(variant="stamps")
+    S = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    S.mbok_gemv.argtypes = [vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp]
+    S.mbok_gemv.restype = i
+    S.mbok_debug_phase_stamps.argtypes = [vp, sz, vp, sz]
+    S.mbok_debug_phase_reset.argtypes = [i]
+    K, M, N, L = (int(v) for v in spec.split(","))
+    assert 2 <= L <= 64
+    dev = torch.device("cuda:0")
+    packed, alphas, xs = build_layers(torch, mb, wl, K, M, N, L, dev, 4242)
+    y = torch.empty(1, M, dtype=torch.float32, device=dev)
+    ws = mb.zeros_workspace(K, M, N, 1, dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def chain():
+        for l in range(L):
+            st = S.mbok_gemv(packed[l].data_ptr(), alphas[l].data_ptr(), K, M, N, 128, xs[l].data_ptr(),
+                             mb.BF16, 1, y.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            assert st == 0, st
+
+    with torch.cuda.stream(stream):
+        chain()   # eager: kernel attributes set outside the capture
+    torch.cuda.synchronize()
+    assert S.mbok_debug_phase_reset(1) == 0   # the capture takes slots 0 .. L-1
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        chain()
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            graph.replay()
+    torch.cuda.synchronize()
+    assert S.mbok_debug_phase_reset(0) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    per_layer_us = e0.elapsed_time(e1) * 1e3 / L
+    main = np.zeros((64, 1024, 5), dtype=np.uint64)
+    comb = np.zeros((64, 1024, 3), dtype=np.uint64)
+    assert S.mbok_debug_phase_stamps(main.ctypes.data, main.nbytes, comb.ctypes.data, comb.nbytes) == 0
+    del graph
+    nm = int((main[0, :, 0] > 0).sum())
+    nc = int((comb[0, :, 0] > 0).sum())
+    terms = {k: [] for k in ("handoff_in", "x_tables", "loop", "drain", "handoff_mid", "combine", "period")}
+    spread = {k: [] for k in ("main_wait_spread", "main_tables_spread", "main_end_spread", "combine_start_spread",
+                              "combine_wait_spread", "combine_cta_work", "combine_end_spread")}
+    for l in range(1, L):
+        m = main[l, :nm].astype(np.int64)
+        c = comb[l, :nc].astype(np.int64)
+        cp = comb[l - 1, :nc].astype(np.int64)
+        prev_end = cp[:, 2].max()
+        v = {"handoff_in": m[:, 1].min() - prev_end,
+             "x_tables": m[:, 2].max() - m[:, 1].min(),
+             "loop": m[:, 3].max() - m[:, 2].max(),
+             "drain": m[:, 4].max() - m[:, 3].max(),
+             "handoff_mid": c[:, 1].min() - m[:, 4].max(),
+             "combine": c[:, 2].max() - c[:, 1].min(),
+             "period": c[:, 2].max() - prev_end}
+        for k, x in v.items():
+            terms[k].append(x / 1000.0)
+        d = {"main_wait_spread": m[:, 1].max() - m[:, 1].min(),
+             "main_tables_spread": m[:, 2].max() - m[:, 2].min(),
+             "main_end_spread": m[:, 4].max() - m[:, 4].min(),
+             "combine_start_spread": c[:, 0].max() - c[:, 0].min(),
+             "combine_wait_spread": c[:, 1].max() - c[:, 1].min(),
+             "combine_cta_work": float(np.median(c[:, 2] - c[:, 1])),
+             "combine_end_spread": c[:, 2].max() - c[:, 2].min()}
+        for k, x in d.items():
+            spread[k].append(x / 1000.0)
+    med = {k: statistics.median(x) for k, x in terms.items()}
+    out = {"phase_profile": f"K={K} {M}x{N} batch 1, {L} layers, graph replay",
+           "main_ctas": nm, "combine_ctas": nc, "layer_us_events": round(per_layer_us, 3),
+           "median_us": {k: round(x, 3) for k, x in med.items()},
+           "share_of_period": {k: round(med[k] / med["period"], 3) for k in med if k != "period"},
+           "spread_median_us": {k: round(statistics.median(x), 3) for k, x in spread.items()}}
+    print(json.dumps(out))
+
+
 def main():
     a = args_parse()
+    if a.phase_profile:
+        phase_profile(a.phase_profile)
+        return
     if a.profile_gemv:
         profile_gemv(a.profile_gemv)
         return

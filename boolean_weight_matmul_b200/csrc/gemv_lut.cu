@@ -39,7 +39,38 @@
 // bit of a kernel and negating its scales reproduces y bit for bit.
 #include "lut_common.cuh"
 
+#ifdef MBOK_PHASE_STAMPS
+#include <atomic>
+#endif
+
 namespace mbok {
+
+// Phase stamps, compiled only into the profiling build (MBOK_PHASE_STAMPS):
+// per CTA, globaltimer readings at the phase boundaries of a decode layer --
+// main kernel: start, dependency wait returned, tables built, last warp out
+// of the streaming loop, last warp's copies drained; combine kernel: start,
+// dependency wait returned, end -- in one of kStampSlots slots per launch.
+// They only record time: the kernels do the same work as without them.
+#ifdef MBOK_PHASE_STAMPS
+constexpr int kStampSlots = 64, kStampCtas = 1024;
+__device__ unsigned long long g_main_stamps[kStampSlots][kStampCtas][5];
+__device__ unsigned long long g_combine_stamps[kStampSlots][kStampCtas][3];
+__device__ __forceinline__ unsigned long long stamp_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+#define MBOK_MAIN_STAMP(slot, pt) \
+  do { if (blockIdx.x < kStampCtas) g_main_stamps[(slot) % kStampSlots][blockIdx.x][pt] = stamp_now(); } while (0)
+#define MBOK_MAIN_STAMP_LAST(slot, pt) \
+  do { if (blockIdx.x < kStampCtas) atomicMax(&g_main_stamps[(slot) % kStampSlots][blockIdx.x][pt], stamp_now()); } while (0)
+#define MBOK_COMBINE_STAMP(slot, pt) \
+  do { if (blockIdx.x < kStampCtas) g_combine_stamps[(slot) % kStampSlots][blockIdx.x][pt] = stamp_now(); } while (0)
+#else
+#define MBOK_MAIN_STAMP(slot, pt) ((void)0)
+#define MBOK_MAIN_STAMP_LAST(slot, pt) ((void)0)
+#define MBOK_COMBINE_STAMP(slot, pt) ((void)0)
+#endif
 
 constexpr int kSlabCols = 512;                  // columns per slab (32 lanes x 16)
 constexpr int kUnitsPerSlab = kSlabCols / kUnit;
@@ -71,6 +102,7 @@ struct GemvParams {
   int nslab, cps;
   int nk;              // kernels handled by separate CTAs: 1 (grouped form) or K (rank-1 form)
   int weights_static;  // bits and scales may be read before the grid dependency wait
+  int stamp_slot;      // profiling build only: this launch's phase-stamp slot
 };
 
 // ---------------------------------------------------------------------------
@@ -219,6 +251,7 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   using G = StageGeom<K>;
   extern __shared__ __align__(1024) unsigned char smem[];
   unsigned char* tab = smem;
+  if (threadIdx.x == 0) MBOK_MAIN_STAMP(p.stamp_slot, 0);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nvs = SV ? p.nslab * p.nk : p.nslab;   // (slab, kernel) CTAs per row range
@@ -264,6 +297,7 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   // x, the workspace and (unless static) the weights may be written by the
   // previous grid: wait for it.
   grid_dependency_wait();
+  if (threadIdx.x == 0) MBOK_MAIN_STAMP(p.stamp_slot, 1);
 
   // x first: its load must not queue behind this warp's weight copies.
   float xv[8];
@@ -288,6 +322,7 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   }
   build_tables(tab, xv, warp, lane);
   __syncthreads();
+  if (threadIdx.x == 0) MBOK_MAIN_STAMP(p.stamp_slot, 2);
 
   for (int t = 0; t < n_mine; ++t) {
     unsigned char* st = ring + (t % kDepth) * G::kBytes;
@@ -322,7 +357,9 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
       }
     }
   }
+  if (lane == 0) MBOK_MAIN_STAMP_LAST(p.stamp_slot, 3);
   cp_async_wait<0>();
+  if (lane == 0) MBOK_MAIN_STAMP_LAST(p.stamp_slot, 4);
   // With several CTAs per row range the partials are combined by
   // gemv_combine_kernel, launched right behind this grid.
 }
@@ -358,6 +395,35 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_multi_kernel(const 
   }
 }
 
+// Sum of the n partials of one row, part[t * stride] for t < n, added in t
+// order.  With more than 8 partials each batch of 16 loads is issued before
+// any of its adds, so a row waits for one L2 round trip per 16 partials
+// rather than one per partial (measured: 7B down, 22 slabs, 8.5 -> 8.0 us per
+// layer; 13B down, 27 slabs, 15.7 -> 15.3 us); with 8 or fewer the plain
+// loop measured as fast or faster.  The sum is the same left-to-right sum
+// either way.
+__device__ __forceinline__ float sum_partials(const float* __restrict__ part, size_t stride, int n) {
+  constexpr int kBatch = 16;
+  float sum = 0.f;
+  if (n <= 8) {
+    for (int t = 0; t < n; ++t) sum += __ldcg(part + size_t(t) * stride);
+    return sum;
+  }
+  for (int t0 = 0; t0 < n; t0 += kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) v[u] = t0 + u < n ? __ldcg(part + size_t(t0 + u) * stride) : 0.f;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (t0 + u < n) sum += v[u];
+  }
+  return sum;
+}
+
+// Threads per CTA of the combine grids: small CTAs spread the rows over
+// many SMs.
+constexpr int kCombineThreads = 64;
+
 struct CombineMultiParams {
   const float* partial[kMaxSegments];   // matrix s: [nslab][O_s * 8]
   int row0[kMaxSegments + 1];           // first output row of matrix s; row0[nseg] = total rows
@@ -367,7 +433,7 @@ struct CombineMultiParams {
 
 // y[R] for the concatenated outputs: the matrix s that row R falls in, then
 // its slabs' partials in slab order (as gemv_combine_kernel).
-__global__ void __launch_bounds__(256) gemv_combine_multi_kernel(const __grid_constant__ CombineMultiParams cm,
+__global__ void __launch_bounds__(kCombineThreads) gemv_combine_multi_kernel(const __grid_constant__ CombineMultiParams cm,
                                                                  float* __restrict__ y) {
   allow_dependents();
   grid_dependency_wait();
@@ -376,24 +442,22 @@ __global__ void __launch_bounds__(256) gemv_combine_multi_kernel(const __grid_co
   int sg = 0;
   while (sg + 1 < cm.nseg && R >= cm.row0[sg + 1]) ++sg;
   const int r = R - cm.row0[sg];
-  const float* part = cm.partial[sg];
-  float sum = 0.f;
-  for (int t = 0; t < cm.nvs; ++t) sum += __ldcg(part + size_t(t) * cm.mpad[sg] + r);
-  y[R] = sum;
+  y[R] = sum_partials(cm.partial[sg] + r, size_t(cm.mpad[sg]), cm.nvs);
 }
 
 // y[r] = sum over the nvs partials of row r, in (kernel, slab) order.  A
 // separate grid, so that no CTA of the main kernel waits on another: its
 // dependency wait returns once every partial of the previous grid is written.
-__global__ void __launch_bounds__(256) gemv_combine_kernel(const float* __restrict__ partial, float* __restrict__ y,
-                                                           int M, int Mpad, int nvs) {
+__global__ void __launch_bounds__(kCombineThreads) gemv_combine_kernel(const float* __restrict__ partial, float* __restrict__ y,
+                                                           int M, int Mpad, int nvs, int stamp_slot) {
+  if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 0);
   allow_dependents();
   grid_dependency_wait();
+  if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 1);
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= M) return;
-  float sum = 0.f;
-  for (int t = 0; t < nvs; ++t) sum += __ldcg(partial + size_t(t) * Mpad + r);
-  y[r] = sum;
+  y[r] = sum_partials(partial + r, size_t(Mpad), nvs);
+  if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 2);
 }
 
 // ---------------------------------------------------------------------------
@@ -427,9 +491,19 @@ static size_t workspace_bytes_for(const Shape& s, int nk) {
 size_t gemv_lut_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, 1); }
 size_t gemv_svid_workspace_bytes(const Shape& s) { return workspace_bytes_for(s, s.K); }
 
+#ifdef MBOK_PHASE_STAMPS
+static std::atomic<int> g_stamp_next{0};   // slot of the next single-matrix launch
+#endif
+
 template <int K, bool XF32, bool SV>
-static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) {
+static cudaError_t launch_k(const GemvParams& p_in, int grid, cudaStream_t stream) {
   using G = StageGeom<K>;
+  GemvParams p = p_in;
+#ifdef MBOK_PHASE_STAMPS
+  p.stamp_slot = g_stamp_next.fetch_add(1) % kStampSlots;
+#else
+  p.stamp_slot = 0;
+#endif
   auto fn = gemv_lut8_kernel<K, XF32, SV>;
   static PerDeviceOnce attr_once;   // the attributes are per device context
   const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), G::kSmem, true);
@@ -449,13 +523,13 @@ static cudaError_t launch_k(const GemvParams& p, int grid, cudaStream_t stream) 
   const int nvs = p.nslab * (SV ? p.nk : 1);
   if (nvs > 1) {
     cudaLaunchConfig_t c2 = {};
-    c2.gridDim = dim3((p.s.M + 255) / 256);
-    c2.blockDim = dim3(256);
+    c2.gridDim = dim3((p.s.M + kCombineThreads - 1) / kCombineThreads);
+    c2.blockDim = dim3(kCombineThreads);
     c2.stream = stream;
     c2.attrs = attr;
     c2.numAttrs = 1;
     e = cudaLaunchKernelEx(&c2, gemv_combine_kernel, static_cast<const float*>(p.partial), p.y, p.s.M,
-                           p.s.O * kOctet, nvs);
+                           p.s.O * kOctet, nvs, p.stamp_slot);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -476,6 +550,7 @@ static GemvParams make_params(const uint8_t* packed, const Shape& s, const void*
   p.cps = pl.cps;
   p.nk = nk;
   p.weights_static = weights_static ? 1 : 0;
+  p.stamp_slot = 0;
   p.partial = pl.nslab * nk > 1 ? static_cast<float*>(workspace) : nullptr;
   return p;
 }
@@ -546,6 +621,7 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
     p.cps = cps;
     p.nk = 1;
     p.weights_static = weights_static ? 1 : 0;
+    p.stamp_slot = 0;
     p.partial = nslab > 1 ? static_cast<float*>(workspace) + poff : nullptr;
     mp.cta0[i] = cta;
     cm.partial[i] = p.partial;
@@ -582,8 +658,8 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
   if (e != cudaSuccess) return e;
   if (nslab > 1) {
     cudaLaunchConfig_t c2 = {};
-    c2.gridDim = dim3((row + 255) / 256);
-    c2.blockDim = dim3(256);
+    c2.gridDim = dim3((row + kCombineThreads - 1) / kCombineThreads);
+    c2.blockDim = dim3(kCombineThreads);
     c2.stream = stream;
     c2.attrs = attr;
     c2.numAttrs = 1;
@@ -606,3 +682,28 @@ cudaError_t launch_gemv_svid(const uint8_t* packed, const uint16_t* s_in, const 
 }
 
 }  // namespace mbok
+
+#ifdef MBOK_PHASE_STAMPS
+// Profiling build only (not part of the C ABI in mbok.h).
+// Copies the stamp arrays out: main [64][1024][5], combine [64][1024][3]
+// unsigned 64-bit nanoseconds; returns a cudaError_t code.
+extern "C" int mbok_debug_phase_stamps(void* main_host, size_t main_bytes, void* combine_host,
+                                       size_t combine_bytes) {
+  cudaError_t e = cudaMemcpyFromSymbol(main_host, mbok::g_main_stamps, main_bytes);
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(combine_host, mbok::g_combine_stamps, combine_bytes);
+  return int(e);
+}
+
+// Zeroes both arrays; with reset_slots != 0 the next launch takes slot 0.
+extern "C" int mbok_debug_phase_reset(int reset_slots) {
+  void* a = nullptr;
+  void* b = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&a, mbok::g_main_stamps);
+  if (e == cudaSuccess) e = cudaMemset(a, 0, sizeof(mbok::g_main_stamps));
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(&b, mbok::g_combine_stamps);
+  if (e == cudaSuccess) e = cudaMemset(b, 0, sizeof(mbok::g_combine_stamps));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (reset_slots) mbok::g_stamp_next.store(0);
+  return int(e);
+}
+#endif

@@ -338,7 +338,7 @@ template <int P, int K, int NT, bool XF32>
 __device__ __forceinline__ void chunk_mmas(const GemvMmaParams& p, const unsigned char* bits, int uq, int g, int n_oct,
                                            const uint32_t b[NT][8], MmaAcc<K, NT>& acc) {
   using G = MmaGeom<K, NT, XF32>;
-  if (NT > 1 || K > 3) {
+  if constexpr (NT > 1 || K > 3) {
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
@@ -355,26 +355,26 @@ __device__ __forceinline__ void chunk_mmas(const GemvMmaParams& p, const unsigne
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc.d[P][k][nt], a[j], b[nt][2 * j], b[nt][2 * j + 1]);
     }
-    return;
+  } else {
+    uint32_t a[K][4][4];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
+      const uint32_t h1 =
+          n_oct > 1 ? *reinterpret_cast<const uint16_t*>(bits + ((K + k) * G::kUnits + uq) * 16 + 2 * g) : 0u;
+      const uint32_t v0 = spread(h0), v1 = spread(h1);
+      a[k][0][0] = sign_pair<0>(v0, p.mul);  a[k][0][1] = sign_pair<0>(v1, p.mul);  a[k][0][2] = sign_pair<2>(v0, p.mul);  a[k][0][3] = sign_pair<2>(v1, p.mul);
+      a[k][1][0] = sign_pair<4>(v0, p.mul);  a[k][1][1] = sign_pair<4>(v1, p.mul);  a[k][1][2] = sign_pair<6>(v0, p.mul);  a[k][1][3] = sign_pair<6>(v1, p.mul);
+      a[k][2][0] = sign_pair<8>(v0, p.mul);  a[k][2][1] = sign_pair<8>(v1, p.mul);  a[k][2][2] = sign_pair<10>(v0, p.mul); a[k][2][3] = sign_pair<10>(v1, p.mul);
+      a[k][3][0] = sign_pair<12>(v0, p.mul); a[k][3][1] = sign_pair<12>(v1, p.mul); a[k][3][2] = sign_pair<14>(v0, p.mul); a[k][3][3] = sign_pair<14>(v1, p.mul);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc.d[P][k][nt], a[k][j], b[nt][2 * j], b[nt][2 * j + 1]);
   }
-  uint32_t a[K][4][4];
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const uint32_t h0 = *reinterpret_cast<const uint16_t*>(bits + (k * G::kUnits + uq) * 16 + 2 * g);
-    const uint32_t h1 =
-        n_oct > 1 ? *reinterpret_cast<const uint16_t*>(bits + ((K + k) * G::kUnits + uq) * 16 + 2 * g) : 0u;
-    const uint32_t v0 = spread(h0), v1 = spread(h1);
-    a[k][0][0] = sign_pair<0>(v0, p.mul);  a[k][0][1] = sign_pair<0>(v1, p.mul);  a[k][0][2] = sign_pair<2>(v0, p.mul);  a[k][0][3] = sign_pair<2>(v1, p.mul);
-    a[k][1][0] = sign_pair<4>(v0, p.mul);  a[k][1][1] = sign_pair<4>(v1, p.mul);  a[k][1][2] = sign_pair<6>(v0, p.mul);  a[k][1][3] = sign_pair<6>(v1, p.mul);
-    a[k][2][0] = sign_pair<8>(v0, p.mul);  a[k][2][1] = sign_pair<8>(v1, p.mul);  a[k][2][2] = sign_pair<10>(v0, p.mul); a[k][2][3] = sign_pair<10>(v1, p.mul);
-    a[k][3][0] = sign_pair<12>(v0, p.mul); a[k][3][1] = sign_pair<12>(v1, p.mul); a[k][3][2] = sign_pair<14>(v0, p.mul); a[k][3][3] = sign_pair<14>(v1, p.mul);
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc.d[P][k][nt], a[k][j], b[nt][2 * j], b[nt][2 * j + 1]);
 }
 
 // One slice: wait for its copies, run this warp's group into d[P]; with
