@@ -395,35 +395,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_lut8_multi_kernel(const 
   }
 }
 
-// Sum of the n partials of one row, part[t * stride] for t < n, added in t
-// order.  With more than 8 partials each batch of 16 loads is issued before
-// any of its adds, so a row waits for one L2 round trip per 16 partials
-// rather than one per partial (measured: 7B down, 22 slabs, 8.5 -> 8.0 us per
-// layer; 13B down, 27 slabs, 15.7 -> 15.3 us); with 8 or fewer the plain
-// loop measured as fast or faster.  The sum is the same left-to-right sum
-// either way.
-__device__ __forceinline__ float sum_partials(const float* __restrict__ part, size_t stride, int n) {
-  constexpr int kBatch = 16;
-  float sum = 0.f;
-  if (n <= 8) {
-    for (int t = 0; t < n; ++t) sum += __ldcg(part + size_t(t) * stride);
-    return sum;
-  }
-  for (int t0 = 0; t0 < n; t0 += kBatch) {
-    float v[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) v[u] = t0 + u < n ? __ldcg(part + size_t(t0 + u) * stride) : 0.f;
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (t0 + u < n) sum += v[u];
-  }
-  return sum;
-}
-
-// Threads per CTA of the combine grids: small CTAs spread the rows over
-// many SMs.
-constexpr int kCombineThreads = 64;
-
 struct CombineMultiParams {
   const float* partial[kMaxSegments];   // matrix s: [nslab][O_s * 8]
   int row0[kMaxSegments + 1];           // first output row of matrix s; row0[nseg] = total rows
@@ -433,7 +404,7 @@ struct CombineMultiParams {
 
 // y[R] for the concatenated outputs: the matrix s that row R falls in, then
 // its slabs' partials in slab order (as gemv_combine_kernel).
-__global__ void __launch_bounds__(kCombineThreads) gemv_combine_multi_kernel(const __grid_constant__ CombineMultiParams cm,
+__global__ void __launch_bounds__(256) gemv_combine_multi_kernel(const __grid_constant__ CombineMultiParams cm,
                                                                  float* __restrict__ y) {
   allow_dependents();
   grid_dependency_wait();
@@ -442,13 +413,16 @@ __global__ void __launch_bounds__(kCombineThreads) gemv_combine_multi_kernel(con
   int sg = 0;
   while (sg + 1 < cm.nseg && R >= cm.row0[sg + 1]) ++sg;
   const int r = R - cm.row0[sg];
-  y[R] = sum_partials(cm.partial[sg] + r, size_t(cm.mpad[sg]), cm.nvs);
+  const float* part = cm.partial[sg];
+  float sum = 0.f;
+  for (int t = 0; t < cm.nvs; ++t) sum += __ldcg(part + size_t(t) * cm.mpad[sg] + r);
+  y[R] = sum;
 }
 
 // y[r] = sum over the nvs partials of row r, in (kernel, slab) order.  A
 // separate grid, so that no CTA of the main kernel waits on another: its
 // dependency wait returns once every partial of the previous grid is written.
-__global__ void __launch_bounds__(kCombineThreads) gemv_combine_kernel(const float* __restrict__ partial, float* __restrict__ y,
+__global__ void __launch_bounds__(256) gemv_combine_kernel(const float* __restrict__ partial, float* __restrict__ y,
                                                            int M, int Mpad, int nvs, int stamp_slot) {
   if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 0);
   allow_dependents();
@@ -456,7 +430,9 @@ __global__ void __launch_bounds__(kCombineThreads) gemv_combine_kernel(const flo
   if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 1);
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= M) return;
-  y[r] = sum_partials(partial + r, size_t(Mpad), nvs);
+  float sum = 0.f;
+  for (int t = 0; t < nvs; ++t) sum += __ldcg(partial + size_t(t) * Mpad + r);
+  y[r] = sum;
   if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 2);
 }
 
@@ -523,8 +499,8 @@ static cudaError_t launch_k(const GemvParams& p_in, int grid, cudaStream_t strea
   const int nvs = p.nslab * (SV ? p.nk : 1);
   if (nvs > 1) {
     cudaLaunchConfig_t c2 = {};
-    c2.gridDim = dim3((p.s.M + kCombineThreads - 1) / kCombineThreads);
-    c2.blockDim = dim3(kCombineThreads);
+    c2.gridDim = dim3((p.s.M + 255) / 256);
+    c2.blockDim = dim3(256);
     c2.stream = stream;
     c2.attrs = attr;
     c2.numAttrs = 1;
@@ -658,8 +634,8 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
   if (e != cudaSuccess) return e;
   if (nslab > 1) {
     cudaLaunchConfig_t c2 = {};
-    c2.gridDim = dim3((row + kCombineThreads - 1) / kCombineThreads);
-    c2.blockDim = dim3(kCombineThreads);
+    c2.gridDim = dim3((row + 255) / 256);
+    c2.blockDim = dim3(256);
     c2.stream = stream;
     c2.attrs = attr;
     c2.numAttrs = 1;
