@@ -74,13 +74,6 @@ struct TcParams {
   int T;
   int n_tile;       // tokens per CTA tile (multiple of 16, <= kTcTokens)
   uint32_t idesc;   // instruction descriptor for N = n_tile
-  // Powers of two for the unpack's left shifts, read from the parameters so
-  // that they stay integer multiply-adds (FMA pipe) instead of becoming
-  // shifts on the ALU pipe, which the selection's logic ops already load:
-  // mul[i] = 2^(15 - 2i) (sign bits of column pair i to bits 15 and 31),
-  // sh = {2, 256, 4, 512} (the index-word placements).
-  uint32_t mul[8];
-  uint32_t sh[4];
 };
 
 // ---------------------------------------------------------------------------
@@ -119,8 +112,8 @@ __device__ __forceinline__ uint32_t tc_pack_bf16x2(float lo, float hi) {
 // where the bit of kernel 0 is 0.  u = h | (h << 15) holds bit b at b and at
 // 15 + b, so one left shift by 15 - 2i puts bit 2i at 15 and bit 2i+1 at 31.
 template <int I>
-__device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t lev, const uint32_t* mul) {
-  const uint32_t s = u * mul[I];   // u << (15 - 2I)
+__device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t lev) {
+  const uint32_t s = u << (15 - 2 * I);
   uint32_t r;
   // r = (~s & 0x80008000) ^ lev
   asm("lop3.b32 %0, %1, %2, %3, 0xA6;\n" : "=r"(r) : "r"(s), "r"(0x80008000u), "r"(lev));
@@ -129,13 +122,9 @@ __device__ __forceinline__ uint32_t tc_signed_pair(uint32_t u, uint32_t lev, con
 
 // Index words of 16 columns from two 16-bit planes (A: index bit 0, B:
 // index bit 1): z[0] covers columns 0..7, z[1] columns 8..15 (layout above).
-// The four masked fields never overlap, so the sums are the bitwise ors.
-__device__ __forceinline__ void tc_index_word(uint32_t A, uint32_t B, const uint32_t* sh, uint32_t& z) {
-  z = (A & 0x55u) * sh[0] + (A & 0xAAu) * sh[1] + (B & 0x55u) * sh[2] + (B & 0xAAu) * sh[3];
-}
-__device__ __forceinline__ void tc_index_words(uint32_t A, uint32_t B, const uint32_t* sh, uint32_t z[2]) {
-  tc_index_word(A, B, sh, z[0]);
-  tc_index_word(A >> 8, B >> 8, sh, z[1]);
+__device__ __forceinline__ void tc_index_words(uint32_t A, uint32_t B, uint32_t z[2]) {
+  z[0] = ((A & 0x55u) << 1) | ((A & 0xAAu) << 8) | ((B & 0x55u) << 2) | ((B & 0xAAu) << 9);
+  z[1] = ((A & 0x5500u) >> 7) | (A & 0xAA00u) | ((B & 0x5500u) >> 6) | ((B & 0xAA00u) << 1);
 }
 
 // prmt.b32 in its default mode, where bit 3 of a selector nibble replicates
@@ -215,16 +204,15 @@ __device__ __forceinline__ void tc_levels(const unsigned char* alpha, int o, int
 // One row x 16 columns: h[k] = the row's 16 bits of kernel k (column b in
 // bit b), P = its levels; out[I] = bf16 pair of columns (2I, 2I+1).
 template <int K>
-__device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_t P[4], const uint32_t* mul,
-                                              const uint32_t* sh, uint32_t out[8]) {
+__device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_t P[4], uint32_t out[8]) {
   const uint32_t u0 = h[0] | (h[0] << 15);
   if (K == 1) {
-#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, P[0], mul);
+#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, P[0]);
     MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
 #undef MBOK_PAIR
   } else if (K == 2) {
     uint32_t z[2];
-    tc_index_words(h[0], h[1], sh, z);
+    tc_index_words(h[0], h[1], z);
 #define MBOK_PAIR(I) out[I] = __byte_perm(P[0], P[1], tc_selector<I>(z));
     MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
 #undef MBOK_PAIR
@@ -232,9 +220,9 @@ __device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_
     // t_k = XNOR(b_k, b_0): the bits relative to kernel 0 (only bits 0..15 are read)
     const uint32_t t1 = ~(h[1] ^ h[0]), t2 = ~(h[2 % K] ^ h[0]);
     uint32_t z[2];
-    tc_index_words(t1, t2, sh, z);
+    tc_index_words(t1, t2, z);
     if (K == 3) {
-#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, __byte_perm(P[0], P[1], tc_selector<I>(z)), mul);
+#define MBOK_PAIR(I) out[I] = tc_signed_pair<I>(u0, __byte_perm(P[0], P[1], tc_selector<I>(z)));
       MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
 #undef MBOK_PAIR
     } else {
@@ -246,8 +234,8 @@ __device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_
     const uint32_t sel = tc_selector<I>(z);                                    \
     const uint32_t lo = __byte_perm(P[0], P[1], sel);                          \
     const uint32_t hi = __byte_perm(P[2], P[3], sel);                          \
-    const uint32_t m = tc_prmt(u3 * mul[I], 0u, 0xBB99u);                      \
-    out[I] = tc_signed_pair<I>(u0, (hi & m) | (lo & ~m), mul);                 \
+    const uint32_t m = tc_prmt(u3 << (15 - 2 * I), 0u, 0xBB99u);               \
+    out[I] = tc_signed_pair<I>(u0, (hi & m) | (lo & ~m));                      \
   }
       MBOK_PAIR(0) MBOK_PAIR(1) MBOK_PAIR(2) MBOK_PAIR(3) MBOK_PAIR(4) MBOK_PAIR(5) MBOK_PAIR(6) MBOK_PAIR(7)
 #undef MBOK_PAIR
@@ -260,8 +248,7 @@ __device__ __forceinline__ void tc_unpack_row(const uint32_t h[K], const uint32_
 // come from the stage's TMA-loaded copy, [octet][k][unit][row] halfwords.
 template <int K, bool SPLIT>
 __device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, const uint32_t P[4],
-                                                    const uint32_t L[4], const uint32_t* mul, const uint32_t* sh,
-                                                    unsigned char* wtile, int tid) {
+                                                    const uint32_t L[4], unsigned char* wtile, int tid) {
   const int r = tid >> 2, u = tid & 3;
   const int o = r >> 3, i = r & 7;
   uint32_t h[K], out[8];
@@ -272,13 +259,13 @@ __device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, c
   // 8 threads of a store phase hold 2 rows of opposite parity x 4 units, i.e.
   // 8 distinct chunks.
   const int c0 = (2 * u) ^ (r & 7), c1 = (2 * u + 1) ^ (r & 7);
-  tc_unpack_row<K>(h, P, mul, sh, out);
+  tc_unpack_row<K>(h, P, out);
   unsigned char* line = wtile + r * 128;
   *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
   *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
   if (SPLIT) {
     // the same selection from the residual levels, into the second tile
-    tc_unpack_row<K>(h, L, mul, sh, out);
+    tc_unpack_row<K>(h, L, out);
     line += kTcWBytes;
     *reinterpret_cast<uint4*>(line + c0 * 16) = make_uint4(out[0], out[1], out[2], out[3]);
     *reinterpret_cast<uint4*>(line + c1 * 16) = make_uint4(out[4], out[5], out[6], out[7]);
@@ -410,7 +397,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j)
-          tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], p.mul, p.sh, st + kTcXBytes,
+          tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], st + kTcXBytes,
                                         tid + j * kTcUnpackWarps * 32);
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
         tc_arrive(&full_w[s]);
@@ -579,8 +566,6 @@ cudaError_t launch_gemm_tc(const uint8_t* packed, const uint16_t* alpha, const S
   p.T = T;
   p.n_tile = n_tile;
   p.idesc = tc_idesc(n_tile);
-  for (int i = 0; i < 8; ++i) p.mul[i] = 1u << (15 - 2 * i);
-  p.sh[0] = 2u; p.sh[1] = 256u; p.sh[2] = 4u; p.sh[3] = 512u;
   switch (s.K) {
     case 1: return split ? launch_tc_k<1, true>(xm, bm, am, p, stream) : launch_tc_k<1, false>(xm, bm, am, p, stream);
     case 2: return split ? launch_tc_k<2, true>(xm, bm, am, p, stream) : launch_tc_k<2, false>(xm, bm, am, p, stream);
