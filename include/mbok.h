@@ -281,15 +281,17 @@ int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* con
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);
 
-/* Whether the lookup GEMV kernels may read their weights (packed bits and
- * scales) before waiting for the preceding launch in the stream.  GEMV
- * launches use programmatic dependent launch: a GEMV may start while the
- * kernel before it finishes, if that kernel signalled early
- * (griddepcontrol.launch_dependents); everything it reads after its wait is
- * ordered after that kernel.  With on = 1 (the default) the first weight
- * tiles are copied into shared memory before the wait, hiding their DRAM
- * latency behind the preceding kernel's tail; activations, outputs and the
- * workspace are always touched after the wait.  This is safe unless a kernel
+/* Whether the GEMV kernels may read their weights (packed bits and scales)
+ * before waiting for the preceding launch in the stream.  GEMV launches use
+ * programmatic dependent launch: a GEMV may start while the kernel before it
+ * finishes, if that kernel signalled early (griddepcontrol.launch_dependents);
+ * everything it reads after its wait is ordered after that kernel.  With
+ * on = 1 (the default) the first weight tiles are copied into shared memory
+ * before the wait, hiding their DRAM latency behind the preceding kernel's
+ * tail -- by the tensor-core kernel always, by the lookup kernels for
+ * launches of up to 16 MB of packed bits (larger launches measured faster
+ * with only their L2 prefetch ahead of the wait); activations, outputs and
+ * the workspace are always touched after the wait.  This is safe unless a kernel
  * that signals early writes the weights right before a GEMV -- no kernel of
  * this library does (the ones that write weights never signal early, so a
  * GEMV after them starts only when they are complete).  on = 0 keeps every
