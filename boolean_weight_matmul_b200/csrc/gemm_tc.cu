@@ -276,6 +276,53 @@ __device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, c
 // The kernel
 // ---------------------------------------------------------------------------
 
+// Drain part of one accumulator tile to Y: this warp's TMEM lane quarter q
+// (rows 32q .. 32q+31 of each 128-row half) and the tile's 16-column chunks
+// first, first + stride, ... (chunk j: half j / cph, columns 16 (j % cph)),
+// loaded kTcDrainBatch at a time per tcgen05.wait::ld.
+constexpr int kTcDrainBatch = 1;
+__device__ __forceinline__ void tc_drain(const TcParams& p, uint32_t tmem, int tile, int row_tiles, int q, int lane,
+                                         int first, int stride) {
+  const int cph = p.n_tile / 16;   // n_tile is a multiple of 16 (the MMA's N)
+  const int nch = 2 * cph;
+  const int t0 = (tile / row_tiles) * p.n_tile;
+  const int rbase = (tile % row_tiles) * kTcRows + 32 * q + lane;
+  for (int j0 = first; j0 < nch; j0 += kTcDrainBatch * stride) {
+    uint32_t v[kTcDrainBatch][16];
+#pragma unroll
+    for (int u = 0; u < kTcDrainBatch; ++u) {
+      const int j = j0 + u * stride;
+      if (j < nch) {
+        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t((j / cph) * 256 + (j % cph) * 16);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+            : "=r"(v[u][0]), "=r"(v[u][1]), "=r"(v[u][2]), "=r"(v[u][3]), "=r"(v[u][4]), "=r"(v[u][5]),
+              "=r"(v[u][6]), "=r"(v[u][7]), "=r"(v[u][8]), "=r"(v[u][9]), "=r"(v[u][10]), "=r"(v[u][11]),
+              "=r"(v[u][12]), "=r"(v[u][13]), "=r"(v[u][14]), "=r"(v[u][15])
+            : "r"(taddr));
+      }
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+    for (int u = 0; u < kTcDrainBatch; ++u) {
+      const int j = j0 + u * stride;
+      const int r = rbase + (j / cph) * kTcHalf;
+      if (j < nch && r < p.s.M) {
+        const int c = t0 + (j % cph) * 16;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          if (c + jj < p.T)
+            p.Y[size_t(c + jj) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[u][jj])));
+        }
+      }
+    }
+  }
+}
+
+// Warps that drain the CTA's last tile: the 16 unpack warps, idle by then,
+// join the 4 epilogue warps (five per TMEM lane quarter).
+constexpr int kTcLastDrainWarps = kTcUnpackWarps + 4;
+
 template <int K, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
@@ -403,6 +450,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         tc_arrive(&full_w[s]);
       }
     }
+    // The CTA's last tile: help the epilogue warps drain it.
+    const int n_mine = blockIdx.x < ntiles ? (ntiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+    if (ok && n_mine > 0) {
+      if (!tc_wait(&tfull[0], unsigned(n_mine - 1) & 1u)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        tc_drain(p, tmem, int(blockIdx.x) + (n_mine - 1) * int(gridDim.x), row_tiles, warp & 3, lane,
+                 (warp - 2) >> 2, kTcLastDrainWarps / 4);
+      }
+    }
   } else {
     // ---- epilogue warps: TMEM quarter (warp & 3) of both row halves ----
     const int quarter = warp & 3;
@@ -410,31 +468,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
       if (!tc_wait(&tfull[0], unsigned(i) & 1u)) { ok = false; break; }
       tc_fence_after();
-      const int t0 = (tile / row_tiles) * p.n_tile;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int r = (tile % row_tiles) * kTcRows + h * kTcHalf + 32 * quarter + lane;
-#pragma unroll 1
-        for (int c = 0; c < p.n_tile; c += 16) {
-          uint32_t v[16];
-          const uint32_t taddr = tmem + (uint32_t(32 * quarter) << 16) + uint32_t(h * 256 + c);
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                "=r"(v[15])
-              : "r"(taddr));
-          asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-          if (r < p.s.M) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int t = t0 + c + j;
-              if (t < p.T)
-                p.Y[size_t(t) * p.s.M + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
-            }
-          }
-        }
-      }
+      const bool last = tile + int(gridDim.x) >= ntiles;
+      if (last)   // shared with the unpack warps: every fifth chunk of this quarter
+        tc_drain(p, tmem, tile, row_tiles, quarter, lane, (warp - 2) >> 2, kTcLastDrainWarps / 4);
+      else
+        tc_drain(p, tmem, tile, row_tiles, quarter, lane, 0, 1);
       tc_fence_before();
       tc_arrive(&tempty[0]);
     }
