@@ -332,12 +332,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   using G = TcGeom<SPLIT>;
   constexpr int kTcStages = G::kStages;
   constexpr int kTcStageBytes = G::kStageBytes;
-  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // stage's TMA data landed
+  uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // stage's X tile landed
   uint64_t* full_w = full_x + kTcStages;   // stage's W tile unpacked
   uint64_t* empty = full_w + kTcStages;    // stage's MMAs done
   uint64_t* tfull = empty + kTcStages;     // accumulator b holds a finished tile
   uint64_t* tempty = tfull + 2;            // accumulator b drained by the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* full_b = tempty + 2;           // stage's bits and scales landed (issued first: the unpack needs only them)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_b + kTcStages);
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -348,6 +349,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       tc_mbar_init(&full_x[s], 1);
+      tc_mbar_init(&full_b[s], 1);
       tc_mbar_init(&full_w[s], kTcUnpackWarps * 32);
       tc_mbar_init(&empty[s], 1);
     }
@@ -382,11 +384,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
           const int s = g % kTcStages;
           if (g >= kTcStages && !tc_wait(&empty[s], unsigned((g / kTcStages) - 1) & 1u)) { ok = false; break; }
           unsigned char* st = smem + s * kTcStageBytes;
-          tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2 + kTcOctets * K * (kTcBitsRow * kOctet + 16));
-          tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
-          tc_tma_load_2d(st + G::kBitsOff, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_x[s]);
+          tc_arrive_expect_tx(&full_b[s], kTcOctets * K * (kTcBitsRow * kOctet + 16));
+          tc_tma_load_2d(st + G::kBitsOff, &bmap, kb * kTcBitsRow * kOctet, (r0 / kOctet) * K, &full_b[s]);
           tc_tma_load_2d(st + G::kAlphaOff, &amap, ((kb * kTcBK) / kGroup) * K * kOctet,
-                         r0 / kOctet, &full_x[s]);
+                         r0 / kOctet, &full_b[s]);
+          tc_arrive_expect_tx(&full_x[s], unsigned(p.n_tile) * kTcBK * 2);
+          tc_tma_load_2d(st, &xmap, kb * kTcBK, t0, &full_x[s]);
         }
       }
     }
@@ -430,8 +433,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < nkb; ++kb, ++g) {
         const int s = g % kTcStages;
-        // the stage's TMA loads landing also means its previous MMAs are done
-        if (!tc_wait(&full_x[s], unsigned(g / kTcStages) & 1u)) { ok = false; break; }
+        // the stage's bits landing also means its previous MMAs are done (the
+        // slot is refilled only after them), so its W tile may be written
+        if (!tc_wait(&full_b[s], unsigned(g / kTcStages) & 1u)) { ok = false; break; }
         unsigned char* st = smem + s * kTcStageBytes;
         // a 128-column group spans two 64-column stages: its levels are
         // formed on the first and kept for the second
@@ -488,6 +492,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     for (int s = 0; s < kTcStages; ++s) {
       (void)tc_wait(&full_x[s], 0u, kTcDrainNs);
       (void)tc_wait(&full_x[s], 1u, kTcDrainNs);
+      (void)tc_wait(&full_b[s], 0u, kTcDrainNs);
+      (void)tc_wait(&full_b[s], 1u, kTcDrainNs);
       (void)tc_wait(&empty[s], 0u, kTcDrainNs);
       (void)tc_wait(&empty[s], 1u, kTcDrainNs);
     }
