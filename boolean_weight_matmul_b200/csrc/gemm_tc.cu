@@ -287,6 +287,9 @@ __device__ __forceinline__ void tc_drain(const TcParams& p, uint32_t tmem, int t
   const int nch = 2 * cph;
   const int t0 = (tile / row_tiles) * p.n_tile;
   const int rbase = (tile % row_tiles) * kTcRows + 32 * q + lane;
+  // Row pairs stored as one 4-byte bf16 pair: needs an even row count (every
+  // pair then lies inside Y's rows and stays 4-byte aligned) and an aligned Y.
+  const bool pairs = (p.s.M % 2) == 0 && (reinterpret_cast<uintptr_t>(p.Y) % 4) == 0;
   for (int j0 = first; j0 < nch; j0 += kTcDrainBatch * stride) {
     uint32_t v[kTcDrainBatch][16];
 #pragma unroll
@@ -306,9 +309,26 @@ __device__ __forceinline__ void tc_drain(const TcParams& p, uint32_t tmem, int t
 #pragma unroll
     for (int u = 0; u < kTcDrainBatch; ++u) {
       const int j = j0 + u * stride;
+      if (j >= nch) continue;
       const int r = rbase + (j / cph) * kTcHalf;
-      if (j < nch && r < p.s.M) {
-        const int c = t0 + (j % cph) * 16;
+      const int c = t0 + (j % cph) * 16;
+      if (pairs) {
+        // Lanes 2i and 2i+1 hold rows r, r+1: after one exchange per token the
+        // even lane has both rows of tokens 0..7 and the odd lane both rows of
+        // tokens 8..15, each stored as one bf16 pair (r0 = the even row).
+        const bool odd = lane & 1;
+        const int r0 = r & ~1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t mine = odd ? v[u][i] : v[u][8 + i];
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          const float lo = __uint_as_float(odd ? other : v[u][i]);        // row r0
+          const float hi = __uint_as_float(odd ? v[u][8 + i] : other);    // row r0 + 1
+          const int t = c + (odd ? 8 + i : i);
+          if (r0 < p.s.M && t < p.T)
+            *reinterpret_cast<uint32_t*>(p.Y + size_t(t) * p.s.M + r0) = tc_pack_bf16x2(lo, hi);
+        }
+      } else if (r < p.s.M) {
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           if (c + jj < p.T)
