@@ -353,12 +353,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   constexpr int kTcStages = G::kStages;
   constexpr int kTcStageBytes = G::kStageBytes;
   uint64_t* full_x = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);   // stage's X tile landed
-  uint64_t* full_w = full_x + kTcStages;   // stage's W tile unpacked
+  uint64_t* full_w = full_x + kTcStages;   // stage's W tile unpacked (split: its rows 0..127)
   uint64_t* empty = full_w + kTcStages;    // stage's MMAs done
   uint64_t* tfull = empty + kTcStages;     // accumulator b holds a finished tile
   uint64_t* tempty = tfull + 2;            // accumulator b drained by the epilogue
   uint64_t* full_b = tempty + 2;           // stage's bits and scales landed (issued first: the unpack needs only them)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_b + kTcStages);
+  uint64_t* full_w1 = full_b + kTcStages;  // split only: stage's W rows 128..255 unpacked
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_w1 + kTcStages);
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -371,6 +372,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       tc_mbar_init(&full_x[s], 1);
       tc_mbar_init(&full_b[s], 1);
       tc_mbar_init(&full_w[s], kTcUnpackWarps * 32);
+      tc_mbar_init(&full_w1[s], kTcUnpackWarps * 32);
       tc_mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -423,20 +425,38 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int s = g % kTcStages;
           const unsigned ph = unsigned(g / kTcStages) & 1u;
-          if (!tc_wait(&full_x[s], ph) || !tc_wait(&full_w[s], ph)) { ok = false; break; }
-          tc_fence_after();
+          if (!tc_wait(&full_x[s], ph)) { ok = false; break; }
           const uint32_t xs = tc_smem(smem + s * kTcStageBytes);
           const uint32_t ws = xs + kTcXBytes;
-#pragma unroll
-          for (int kk = 0; kk < kTcBK / 16; ++kk) {
-            const uint64_t bdesc = tc_desc_sw128(xs + kk * 32);
+          if constexpr (SPLIT) {
+            // Each 128-row half of W (both its tiles) is issued as soon as it
+            // is unpacked: measured faster for the split (106.0 -> 101.8 us).
+            // The single tile keeps the k-outer order over both halves.
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + h * (kTcHalf * 128) + kk * 32), bdesc, p.idesc,
-                     (kb > 0 || kk > 0) ? 1u : 0u);
-              if (SPLIT)   // the residual tile into the same accumulator
+              if (!tc_wait(h == 0 ? &full_w[s] : &full_w1[s], ph)) { ok = false; break; }
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kTcBK / 16; ++kk) {
+                const uint64_t bdesc = tc_desc_sw128(xs + kk * 32);
+                tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + h * (kTcHalf * 128) + kk * 32), bdesc, p.idesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
+                // the residual tile into the same accumulator
                 tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + kTcWBytes + h * (kTcHalf * 128) + kk * 32), bdesc,
                        p.idesc, 1u);
+              }
+            }
+            if (!ok) break;
+          } else {
+            if (!tc_wait(&full_w[s], ph)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTcBK / 16; ++kk) {
+              const uint64_t bdesc = tc_desc_sw128(xs + kk * 32);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tc_mma(tmem + uint32_t(h * 256), tc_desc_sw128(ws + h * (kTcHalf * 128) + kk * 32), bdesc, p.idesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit(&empty[s]);
@@ -457,21 +477,39 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         // slot is refilled only after them), so its W tile may be written
         if (!tc_wait(&full_b[s], unsigned(g / kTcStages) & 1u)) { ok = false; break; }
         unsigned char* st = smem + s * kTcStageBytes;
-        // a 128-column group spans two 64-column stages: its levels are
-        // formed on the first and kept for the second
-        if ((kb & 1) == 0) {
+        // Pass j unpacks rows 128 j .. 128 j + 127.  A 128-column group spans
+        // two 64-column stages: its levels are formed on the first and kept
+        // for the second.  The split releases each half to the MMA thread as
+        // soon as it is written (full_w, full_w1); the single tile releases
+        // the whole tile at the end on full_w (a second 512-thread arrival
+        // per stage measured 2 us slower over the GEMM).
+        if constexpr (SPLIT) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const int r = (tid + j * kTcUnpackWarps * 32) >> 2;
-            tc_levels<K, SPLIT>(st + G::kAlphaOff, r >> 3, r & 7, lev[j], res[j]);
+            if ((kb & 1) == 0) {
+              const int r = (tid + j * kTcUnpackWarps * 32) >> 2;
+              tc_levels<K, SPLIT>(st + G::kAlphaOff, r >> 3, r & 7, lev[j], res[j]);
+            }
+            tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], st + kTcXBytes,
+                                          tid + j * kTcUnpackWarps * 32);
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
+            tc_arrive(j == 0 ? &full_w[s] : &full_w1[s]);
           }
-        }
+        } else {
+          if ((kb & 1) == 0) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-          tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], st + kTcXBytes,
-                                        tid + j * kTcUnpackWarps * 32);
-        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
-        tc_arrive(&full_w[s]);
+            for (int j = 0; j < 2; ++j) {
+              const int r = (tid + j * kTcUnpackWarps * 32) >> 2;
+              tc_levels<K, SPLIT>(st + G::kAlphaOff, r >> 3, r & 7, lev[j], res[j]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tc_unpack_from_smem<K, SPLIT>(st + G::kBitsOff, lev[j], res[j], st + kTcXBytes,
+                                          tid + j * kTcUnpackWarps * 32);
+          asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor core reads
+          tc_arrive(&full_w[s]);
+        }
       }
     }
     // The CTA's last tile: help the epilogue warps drain it.
