@@ -19,12 +19,13 @@
 //    copies: per (octet, kernel) one copy per lane (512 contiguous bytes per
 //    warp), plus the octet's 4 groups x K scale vectors.  The main loop has
 //    no block-wide barrier.  Launches use programmatic dependent launch:
-//    before waiting on the previous grid the kernel prefetches its first
-//    octets and its slice of x into L2 and (unless turned off, because a
-//    kernel that lets this grid start early might write the weights) starts
-//    the octets' shared-memory copies; the read of x and every write happen
-//    after the wait.  A chain of layers thus overlaps one launch's tail with
-//    the next launch's weights.
+//    before waiting on the previous grid, a launch of up to 16 MB of packed
+//    bits prefetches its first octets into L2 and (unless turned off,
+//    because a kernel that lets this grid start early might write the
+//    weights) starts the octets' shared-memory copies; every launch
+//    prefetches its slice of x into L2; the read of x and every write happen
+//    after the wait.  A chain of small layers thus overlaps one launch's tail
+//    with the next launch's weights.
 //  * Per (row pair, kernel) a lane does four lookups, one packed fp32x2 add
 //    and one packed fp32x2 FMA with the two rows' fp16 group scales.
 //  * The 32 lanes' partial sums of an octet's 8 rows are combined by a
@@ -79,7 +80,7 @@ constexpr int kGemvThreads = 512;
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kLutBytes = 256 * 256;            // 256 entries x (32 lanes x 2 tables x 4 B)
 constexpr int kDepth = 3;                       // octets in flight per warp
-constexpr int kPrefetchOctets = 16;             // L2 prefetch ahead of the dependency wait, per warp
+constexpr int kPrefetchOctets = 16;             // L2 prefetch ahead of the dependency wait, per warp (launches <= 16 MB)
 
 template <int K>
 struct StageGeom {
@@ -103,6 +104,7 @@ struct GemvParams {
   int nk;              // kernels handled by separate CTAs: 1 (grouped form) or K (rank-1 form)
   int weights_static;  // bits and scales may be read before the grid dependency wait
   int stamp_slot;      // profiling build only: this launch's phase-stamp slot
+  int prefetch_octets; // octets per warp prefetched into L2 before the dependency wait
 };
 
 // ---------------------------------------------------------------------------
@@ -271,11 +273,12 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   const int first = o_begin + warp;
   const int n_mine = first < o_end ? (o_end - first + kGemvWarps - 1) / kGemvWarps : 0;
 
-  // Before the dependency wait: L2 prefetches of this warp's first octets,
-  // and unless the caller turned it off (mbok_gemv_set_static_weights) the
-  // first octets' copies into shared memory as well -- weights are not
-  // written by kernels that let this grid start early.
-  for (int t = 0; t < kPrefetchOctets && t < n_mine; ++t)
+  // Before the dependency wait (launches of up to 16 MB): L2 prefetches of
+  // this warp's first octets, and unless the caller turned it off
+  // (mbok_gemv_set_static_weights) the first octets' copies into shared
+  // memory as well -- weights are not written by kernels that let this grid
+  // start early.
+  for (int t = 0; t < p.prefetch_octets && t < n_mine; ++t)
     prefetch_octet<K, SV>(p, slab, units, groups, first + t * kGemvWarps, kk, lane);
   if (p.weights_static) {
 #pragma unroll
@@ -511,17 +514,20 @@ static cudaError_t launch_k(const GemvParams& p_in, int grid, cudaStream_t strea
   return cudaGetLastError();
 }
 
-// Whether a launch copies its first weight tiles into shared memory before
-// the grid dependency wait (only ever with static weights).  Measured in a
-// chain of layers: it pays for launches of up to ~16 MB of packed bits
-// (q_proj 4.86 vs 5.32 us, 7B down 8.55 vs 9.03 us) and costs on larger ones
-// (fused LLaMA-13B sweep 402 vs 413 tokens/s), where the early copies
-// compete with the previous layer's own streaming.  The L2 prefetch ahead
-// of the wait runs either way.
+// What a launch reads before the grid dependency wait.  Launches of up to
+// 16 MB of packed bits prefetch each warp's first kPrefetchOctets octets into
+// L2 and, with static weights, copy the first tiles into shared memory:
+// measured in a chain of layers, that hides their DRAM latency behind the
+// previous layer's tail (q_proj 4.82 vs 5.26 us/layer without the prefetch,
+// 4.86 vs 5.32 us without the copies).  Larger launches read nothing ahead of
+// the wait: there the early traffic competes with the previous layer's own
+// streaming (7B gate 8.74 -> 8.25 us/layer; fused LLaMA-13B sweep 402 ->
+// 413 tokens/s without the early copies and 413 -> 453 without the prefetch).
 constexpr size_t kEarlyStageMaxBytes = size_t(16) << 20;
 inline bool stage_early(bool weights_static, size_t packed_bytes) {
   return weights_static && packed_bytes <= kEarlyStageMaxBytes;
 }
+inline int prefetch_depth(size_t packed_bytes) { return packed_bytes <= kEarlyStageMaxBytes ? kPrefetchOctets : 0; }
 
 static GemvParams make_params(const uint8_t* packed, const Shape& s, const void* x, float* y, void* workspace,
                               bool weights_static, int nk) {
@@ -539,6 +545,7 @@ static GemvParams make_params(const uint8_t* packed, const Shape& s, const void*
   p.nk = nk;
   p.weights_static = stage_early(weights_static, size_t(s.O) * kOctet * s.K * (s.N / 8)) ? 1 : 0;
   p.stamp_slot = 0;
+  p.prefetch_octets = prefetch_depth(size_t(s.O) * kOctet * s.K * (s.N / 8));
   p.partial = pl.nslab * nk > 1 ? static_cast<float*>(workspace) : nullptr;
   return p;
 }
@@ -613,6 +620,7 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
     p.nk = 1;
     p.weights_static = early ? 1 : 0;
     p.stamp_slot = 0;
+    p.prefetch_octets = prefetch_depth(launch_bytes);
     p.partial = nslab > 1 ? static_cast<float*>(workspace) + poff : nullptr;
     mp.cta0[i] = cta;
     cm.partial[i] = p.partial;

@@ -290,8 +290,8 @@ int mbok_gemv_set_kernel(int kernel);
  * before the wait, hiding their DRAM latency behind the preceding kernel's
  * tail -- by the tensor-core kernel always, by the lookup kernels for
  * launches of up to 16 MB of packed bits (larger launches measured faster
- * with only their L2 prefetch ahead of the wait); activations, outputs and
- * the workspace are always touched after the wait.  This is safe unless a kernel
+ * reading nothing ahead of the wait); activations, outputs and the
+ * workspace are always touched after the wait.  This is safe unless a kernel
  * that signals early writes the weights right before a GEMV -- no kernel of
  * this library does (the ones that write weights never signal early, so a
  * GEMV after them starts only when they are complete).  on = 0 keeps every
