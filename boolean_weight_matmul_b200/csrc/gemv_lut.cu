@@ -433,18 +433,29 @@ __global__ void __launch_bounds__(256) gemv_combine_kernel(const float* __restri
   if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 1);
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= M) return;
-  // The first 8 partials are loaded before any is added, so they cost one L2
-  // round trip (bench, same box: q_proj 4.88 -> 4.68 us per layer); the sum
-  // is the same slab-order sum.  (The same change in the multi-matrix combine
-  // measured slower and is not made there.)
-  float v[8];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) v[t] = t < nvs ? __ldcg(partial + size_t(t) * Mpad + r) : 0.f;
+  // The first partials (8 with up to 8 slabs, else 16) are loaded before any
+  // is added, so they cost one L2 round trip; the sum is the same slab-order
+  // sum.  Measured (bench, same box): 8 wide, q_proj (8 slabs) 4.88 -> 4.68 us
+  // per layer; 16 wide, 7B down (22 slabs) 8.06 -> 7.73 us and the fused
+  // LLaMA-13B sweep (10 and 27 slabs) 455 -> 464 tokens/s, but 5.32 us on
+  // q_proj.  (Batching the multi-matrix combine measured slower there.)
   float sum = 0.f;
+  if (nvs <= 8) {
+    float v[8];
 #pragma unroll
-  for (int t = 0; t < 8; ++t)
-    if (t < nvs) sum += v[t];
-  for (int t = 8; t < nvs; ++t) sum += __ldcg(partial + size_t(t) * Mpad + r);
+    for (int t = 0; t < 8; ++t) v[t] = t < nvs ? __ldcg(partial + size_t(t) * Mpad + r) : 0.f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (t < nvs) sum += v[t];
+  } else {
+    float v[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) v[t] = t < nvs ? __ldcg(partial + size_t(t) * Mpad + r) : 0.f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      if (t < nvs) sum += v[t];
+    for (int t = 16; t < nvs; ++t) sum += __ldcg(partial + size_t(t) * Mpad + r);
+  }
   y[r] = sum;
   if (threadIdx.x == 0) MBOK_COMBINE_STAMP(stamp_slot, 2);
 }
