@@ -416,9 +416,24 @@ __global__ void __launch_bounds__(256) gemv_combine_multi_kernel(const __grid_co
   int sg = 0;
   while (sg + 1 < cm.nseg && R >= cm.row0[sg + 1]) ++sg;
   const int r = R - cm.row0[sg];
-  const float* part = cm.partial[sg];
+  const float* part = cm.partial[sg] + r;
+  const size_t stride = size_t(cm.mpad[sg]);
+  const int nvs = cm.nvs;
   float sum = 0.f;
-  for (int t = 0; t < cm.nvs; ++t) sum += __ldcg(part + size_t(t) * cm.mpad[sg] + r);
+  // As gemv_combine_kernel, but with up to 8 slabs the plain loop: batching
+  // those measured slower here (mixed-K LLaMA-13B sweep 454 -> 437 tokens/s);
+  // 16 at once above 8 slabs took it 454 -> 472.
+  if (nvs <= 8) {
+    for (int t = 0; t < nvs; ++t) sum += __ldcg(part + size_t(t) * stride);
+  } else {
+    float v[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) v[t] = t < nvs ? __ldcg(part + size_t(t) * stride) : 0.f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      if (t < nvs) sum += v[t];
+    for (int t = 16; t < nvs; ++t) sum += __ldcg(part + size_t(t) * stride);
+  }
   y[R] = sum;
 }
 
@@ -438,7 +453,7 @@ __global__ void __launch_bounds__(256) gemv_combine_kernel(const float* __restri
   // sum.  Measured (bench, same box): 8 wide, q_proj (8 slabs) 4.88 -> 4.68 us
   // per layer; 16 wide, 7B down (22 slabs) 8.06 -> 7.73 us and the fused
   // LLaMA-13B sweep (10 and 27 slabs) 455 -> 464 tokens/s, but 5.32 us on
-  // q_proj.  (Batching the multi-matrix combine measured slower there.)
+  // q_proj.  The multi-matrix combine batches only above 8 slabs.
   float sum = 0.f;
   if (nvs <= 8) {
     float v[8];
