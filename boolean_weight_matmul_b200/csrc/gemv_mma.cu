@@ -20,7 +20,7 @@
 //    and added into the output accumulators (fp32 FMA), so the scales are
 //    applied exactly as the method's grouped sum states.
 //  * A CTA owns one 16-row tile (two storage octets) and all N columns.  The
-//    tile's bits and scales stream through a 4-stage shared-memory ring in
+//    tile's bits and scales stream through a ring of up to 8 stages in
 //    1024-column slices: per slice, one bulk asynchronous copy per (octet,
 //    kernel) (the slice is contiguous in storage format 1) and one per octet
 //    for the scales, completing on the stage's mbarrier.  The 8 warps split
@@ -48,7 +48,16 @@ namespace mbok {
 constexpr int kMmaWarps = 8;
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kChunkCols = 64;                      // 4 units, 4 MMAs per kernel
-constexpr int kMmaStages = 4;
+// Ring stages: 4, or for rows of 8 or more slices (N > 7168) 8 where they
+// leave room for three CTAs per SM (228 KB / 3, less each CTA's 1 KB
+// reservation and its static shared memory).  Measured: 7B down (11 slices)
+// b4 17.4 -> 16.4 us, b16 21.0 -> 20.0 us with the deep ring; with 5 slices
+// (LLaMA-13B gate, N = 5120) the extra stages only took L1 room from the
+// activations (b4 31.1 -> 33.2 us), so short rows keep 4.
+constexpr int kMmaShortStages = 4;
+constexpr int kMmaMaxStages = 8;
+constexpr int kMmaDeepMinSlices = 8;
+constexpr int kMmaCtaSmemBudget = 74 * 1024;
 constexpr int kMaxNT = 2;                           // up to 16 columns of B per launch
 constexpr unsigned long long kMmaWaitNs = 1000000000ull;
 constexpr unsigned long long kMmaDrainNs = 200000000ull;
@@ -56,7 +65,7 @@ constexpr unsigned long long kMmaDrainNs = 200000000ull;
 // One ring stage: a slice of kCols columns of the tile's two octets (bits of
 // every kernel, scales).  Activations are read from global memory (they are
 // shared by every CTA and stay in L1/L2), one chunk ahead of their use.
-template <int K, int NT, bool XF32>
+template <int K, int NT, bool XF32, bool DEEP = false>
 struct MmaGeom {
   static constexpr int kCols = 1024;
   static constexpr int kUnits = kCols / kUnit;
@@ -67,7 +76,12 @@ struct MmaGeom {
   static constexpr int kAlpha = 2 * kGroups * K * 16;           // [octet][group][k][8 rows][2 B]
   static constexpr int kStage = kBits + kAlpha;
   static constexpr int kRed = kMmaWarps * NT * 8 * 16 * 4;
-  static constexpr int kSmem = kMmaStages * kStage + kRed;
+  // a power of two (stage index and phase are a mask and a shift): 8 where
+  // it fits the budget (K <= 3), else 4
+  static constexpr int kDeepStages = (kMmaCtaSmemBudget - kRed) / kStage >= kMmaMaxStages ? kMmaMaxStages
+                                                                                          : kMmaShortStages;
+  static constexpr int kStages = DEEP ? kDeepStages : kMmaShortStages;
+  static constexpr int kSmem = kStages * kStage + kRed;
 };
 
 __device__ unsigned int g_gemv_mma_error;
@@ -384,21 +398,21 @@ __device__ __forceinline__ void chunk_mmas(const GemvMmaParams& p, const unsigne
 // deferral), released by every warp one step earlier.  False if a wait gave
 // up.  b0 holds the activations of this warp's chunk 0 in slice sl; b1 is
 // filled with those of chunk 1, and b0 with the next slice's chunk 0.
-template <int P, int K, int NT, bool XF32>
+template <int P, int K, int NT, bool XF32, bool DEEP>
 __device__ __forceinline__ bool mma_slice(const GemvMmaParams& p, MmaCtx& c, MmaAcc<K, NT>& acc, int sl,
                                           uint32_t b0[NT][8], uint32_t b1[NT][8]) {
-  using G = MmaGeom<K, NT, XF32>;
+  using G = MmaGeom<K, NT, XF32, DEEP>;
   constexpr bool kDefer = MmaDefer<K, NT>::value;
   constexpr int kLag = kDefer ? 2 : 1;
   constexpr int stage_bytes = G::kStage;
-  const int st = sl % kMmaStages;
-  const unsigned phase = unsigned(sl / kMmaStages) & 1u;
+  const int st = sl % G::kStages;
+  const unsigned phase = unsigned(sl / G::kStages) & 1u;
   // Every decision below is made warp-uniform (the MMAs are warp-wide).
   bool good = true;
   if (c.warp == 0) {
     if (c.lane == 0 && sl >= kLag && c.issued < c.n_slices) {
-      const int pst = (sl - kLag) % kMmaStages;
-      good = mm_wait(&c.empty[pst], unsigned((sl - kLag) / kMmaStages) & 1u, kMmaWaitNs);
+      const int pst = (sl - kLag) % G::kStages;
+      good = mm_wait(&c.empty[pst], unsigned((sl - kLag) / G::kStages) & 1u, kMmaWaitNs);
       if (good) {
         issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, c.smem + pst * stage_bytes, &c.full[pst]);
         ++c.issued;
@@ -428,7 +442,7 @@ __device__ __forceinline__ bool mma_slice(const GemvMmaParams& p, MmaCtx& c, Mma
   }
   if (kDefer) {
     if (sl >= 1) {
-      const int pst = (sl - 1) % kMmaStages;
+      const int pst = (sl - 1) % G::kStages;
       acc.template flush<MmaDefer<K, NT>::kSets - 1 - P>(c.smem + pst * stage_bytes + G::kBits, w, c.g, c.n_oct,
                                                           G::kGroups);
       __syncwarp();
@@ -446,13 +460,13 @@ __device__ __forceinline__ bool mma_slice(const GemvMmaParams& p, MmaCtx& c, Mma
 // enough to fill three per SM (more warps to hide latency), else 2 (the
 // scheduler would otherwise crowd a small grid onto fewer SMs); 1 for the
 // register-heavy variants with two 8-column tiles and K >= 3.
-template <int K, int NT, bool XF32, int MINB>
+template <int K, int NT, bool XF32, int MINB, bool DEEP>
 __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaParams p) {
-  using G = MmaGeom<K, NT, XF32>;
+  using G = MmaGeom<K, NT, XF32, DEEP>;
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int stage_bytes = G::kStage;
-  float (*red)[NT * 8][16] = reinterpret_cast<float (*)[NT * 8][16]>(smem + kMmaStages * stage_bytes);
-  __shared__ __align__(8) uint64_t full[kMmaStages], empty[kMmaStages];
+  float (*red)[NT * 8][16] = reinterpret_cast<float (*)[NT * 8][16]>(smem + G::kStages * stage_bytes);
+  __shared__ __align__(8) uint64_t full[G::kStages], empty[G::kStages];
   __shared__ int s_abort;
 
   MmaCtx c;
@@ -471,7 +485,7 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
   c.n_slices = (s.N + G::kCols - 1) / G::kCols;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMmaStages; ++i) {
+    for (int i = 0; i < G::kStages; ++i) {
       mm_bar_init(&full[i], 1);
       mm_bar_init(&empty[i], kMmaWarps);
     }
@@ -480,7 +494,7 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
     // Weights that no earlier kernel on the stream writes: the ring's first
     // slices are copied before the dependency wait.
     if (p.weights_static) {
-      for (; c.issued < kMmaStages && c.issued < c.n_slices; ++c.issued)
+      for (; c.issued < G::kStages && c.issued < c.n_slices; ++c.issued)
         issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, smem + c.issued * stage_bytes, &full[c.issued]);
     }
   }
@@ -503,7 +517,7 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
   __syncthreads();   // barrier initialisation visible to all threads
 
   if (threadIdx.x == 0) {
-    for (; c.issued < kMmaStages && c.issued < c.n_slices; ++c.issued)
+    for (; c.issued < G::kStages && c.issued < c.n_slices; ++c.issued)
       issue_slice<K, NT, XF32>(p, c.o0, c.n_oct, c.issued, smem + c.issued * stage_bytes, &full[c.issued]);
   }
 
@@ -520,23 +534,23 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
   int done = 0;   // slices completed
   if (kDefer) {
     for (int sl = 0; sl < c.n_slices; sl += 2) {
-      if (!mma_slice<0, K, NT, XF32>(p, c, acc, sl, b0, b1)) break;
+      if (!mma_slice<0, K, NT, XF32, DEEP>(p, c, acc, sl, b0, b1)) break;
       ++done;
       if (sl + 1 < c.n_slices) {
-        if (!mma_slice<MmaDefer<K, NT>::kSets - 1, K, NT, XF32>(p, c, acc, sl + 1, b0, b1)) break;
+        if (!mma_slice<MmaDefer<K, NT>::kSets - 1, K, NT, XF32, DEEP>(p, c, acc, sl + 1, b0, b1)) break;
         ++done;
       }
     }
     // The last slice's group is still pending; its stage is still held.
     if (done == c.n_slices && c.n_slices >= 1) {
       const int last = c.n_slices - 1;
-      const unsigned char* alph = smem + (last % kMmaStages) * stage_bytes + G::kBits;
+      const unsigned char* alph = smem + (last % G::kStages) * stage_bytes + G::kBits;
       if (last & 1) acc.template flush<MmaDefer<K, NT>::kSets - 1>(alph, c.warp, c.g, c.n_oct, G::kGroups);
       else acc.template flush<0>(alph, c.warp, c.g, c.n_oct, G::kGroups);
     }
   } else {
     for (int sl = 0; sl < c.n_slices; ++sl) {
-      if (!mma_slice<0, K, NT, XF32>(p, c, acc, sl, b0, b1)) break;
+      if (!mma_slice<0, K, NT, XF32, DEEP>(p, c, acc, sl, b0, b1)) break;
       ++done;
     }
   }
@@ -556,7 +570,7 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
     // Wait (bounded) for every copy this CTA issued, then leave without storing.
     if (threadIdx.x == 0) {
       for (int sl = 0; sl < c.issued; ++sl)
-        mm_wait(&full[sl % kMmaStages], unsigned(sl / kMmaStages) & 1u, kMmaDrainNs);
+        mm_wait(&full[sl % G::kStages], unsigned(sl / G::kStages) & 1u, kMmaDrainNs);
     }
     return;
   }
@@ -588,10 +602,10 @@ __global__ void __launch_bounds__(kMmaThreads, MINB) gemv_mma_kernel(GemvMmaPara
 // Host side
 // ---------------------------------------------------------------------------
 
-template <int K, int NT, bool XF32, int MINB>
+template <int K, int NT, bool XF32, int MINB, bool DEEP>
 static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
-  auto fn = gemv_mma_kernel<K, NT, XF32, MINB>;
-  using G = MmaGeom<K, NT, XF32>;
+  auto fn = gemv_mma_kernel<K, NT, XF32, MINB, DEEP>;
+  using G = MmaGeom<K, NT, XF32, DEEP>;
   static PerDeviceOnce attr_once;   // the attribute is per device context
   const cudaError_t ae = set_smem_attr_once(attr_once, reinterpret_cast<const void*>(fn), G::kSmem);
   if (ae != cudaSuccess) return ae;
@@ -610,16 +624,25 @@ static cudaError_t launch_mma_k(const GemvMmaParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int K>
-static cudaError_t launch_mma_nt(const GemvMmaParams& p, bool x_f32, cudaStream_t stream) {
+template <int K, bool DEEP>
+static cudaError_t launch_mma_nt_d(const GemvMmaParams& p, bool x_f32, cudaStream_t stream) {
   const int cols = x_f32 ? 3 * p.nb : p.nb;
   const bool big_grid = (p.s.O + 1) / 2 >= 3 * device_sm_count();
   if (cols <= 8) {
-    if (big_grid) return x_f32 ? launch_mma_k<K, 1, true, 3>(p, stream) : launch_mma_k<K, 1, false, 3>(p, stream);
-    return x_f32 ? launch_mma_k<K, 1, true, 2>(p, stream) : launch_mma_k<K, 1, false, 2>(p, stream);
+    if (big_grid)
+      return x_f32 ? launch_mma_k<K, 1, true, 3, DEEP>(p, stream) : launch_mma_k<K, 1, false, 3, DEEP>(p, stream);
+    return x_f32 ? launch_mma_k<K, 1, true, 2, DEEP>(p, stream) : launch_mma_k<K, 1, false, 2, DEEP>(p, stream);
   }
   constexpr int kMinB2 = K >= 3 ? 1 : 2;
-  return x_f32 ? launch_mma_k<K, 2, true, kMinB2>(p, stream) : launch_mma_k<K, 2, false, kMinB2>(p, stream);
+  return x_f32 ? launch_mma_k<K, 2, true, kMinB2, DEEP>(p, stream)
+               : launch_mma_k<K, 2, false, kMinB2, DEEP>(p, stream);
+}
+
+template <int K>
+static cudaError_t launch_mma_nt(const GemvMmaParams& p, bool x_f32, cudaStream_t stream) {
+  const int slices = (p.s.N + MmaGeom<K, 1, false>::kCols - 1) / MmaGeom<K, 1, false>::kCols;
+  return slices >= kMmaDeepMinSlices ? launch_mma_nt_d<K, true>(p, x_f32, stream)
+                                     : launch_mma_nt_d<K, false>(p, x_f32, stream);
 }
 
 // Self-check of the bounded waits: one warp waits, with the kernels' own wait
