@@ -273,6 +273,21 @@ def test_gemv_tensor_mlp_sampled(name, M, N, batch):
     assert_close(y, y_ref, E, GEMV_REL_L2, f"tensor {name} b{batch}")
 
 
+@pytest.mark.parametrize("K", [1, 2, 3, 4])
+@pytest.mark.parametrize("batch", [3, 12])
+def test_gemv_tensor_long_rows(K, batch):
+    # Rows of 8 or more 1024-column slices take the tensor kernel's deep copy
+    # ring: N = 8320 is nine slices, the last one partial (one 128-column
+    # group); ragged M; one (batch 3) and two (batch 12) 8-column tiles of B;
+    # bf16 and fp32 activations; every output checked.
+    import boolean_weight_matmul_b200 as mb
+    M, N = 72, 8320
+    with mb.gemv_kernel(mb.GEMV_TENSOR):
+        for x_dtype in ("bf16", "f32"):
+            y, y_ref, E = _gemv_case(K, M, N, batch, x_dtype, 6800 + 10 * K + batch, "decaying")
+            assert_close(y, y_ref, E, GEMV_REL_L2, f"tensor long rows K={K} b={batch} {x_dtype}")
+
+
 @pytest.mark.parametrize("kernel", ["lookup", "tensor", "lookup_rows"])
 def test_gemv_kernel_flip_invariance_bitwise(kernel):
     # Negated signs (exact) times negated scales: the same y bit for bit.
