@@ -450,6 +450,7 @@ def _multi_case(Ks, Ms, N, batch, x_dtype, seed):
     ((3, 1), (40, 8), 512, 2, "f32"),                 # one slab: outputs stored directly, two vectors
     ((2,), (300,), 1024, 1, "bf16"),                  # a single matrix
     ((1, 2, 3, 4, 1, 2, 3, 4), (8, 16, 24, 32, 40, 48, 56, 64), 640, 1, "bf16"),   # eight matrices, ragged slab
+    ((3, 1), (40, 24), 9216, 1, "bf16"),              # 18 slabs: the combine's batch of 16 and its remainder
 ])
 def test_gemv_multi_equals_separate_calls(Ks, Ms, N, batch, x_dtype):
     # Each row is computed as in its own matrix's launch (same tables, same
