@@ -280,7 +280,7 @@ __device__ __forceinline__ void tc_unpack_from_smem(const unsigned char* bits, c
 // (rows 32q .. 32q+31 of each 128-row half) and the tile's 16-column chunks
 // first, first + stride, ... (chunk j: half j / cph, columns 16 (j % cph)),
 // loaded kTcDrainBatch at a time per tcgen05.wait::ld.
-constexpr int kTcDrainBatch = 1;
+constexpr int kTcDrainBatch = 1;   // 2 or 3 chunks per wait spilled at the 80-register budget and measured slower
 __device__ __forceinline__ void tc_drain(const TcParams& p, uint32_t tmem, int tile, int row_tiles, int q, int lane,
                                          int first, int stride) {
   const int cph = p.n_tile / 16;   // n_tile is a multiple of 16 (the MMA's N)
@@ -359,7 +359,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   uint64_t* tempty = tfull + 2;            // accumulator b drained by the epilogue
   uint64_t* full_b = tempty + 2;           // stage's bits and scales landed (issued first: the unpack needs only them)
   uint64_t* full_w1 = full_b + kTcStages;  // split only: stage's W rows 128..255 unpacked
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full_w1 + kTcStages);
+  uint64_t* last_full = full_w1 + kTcStages;   // the CTA's last tile is in the accumulator (completes once)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(last_full + 1);
   __shared__ int s_fail;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -379,6 +380,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       tc_mbar_init(&tfull[b], 1);
       tc_mbar_init(&tempty[b], 4 * 32);
     }
+    tc_mbar_init(last_full, 1);
     s_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -512,10 +514,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
       }
     }
-    // The CTA's last tile: help the epilogue warps drain it.
+    // The CTA's last tile: help the epilogue warps drain it.  The epilogue
+    // warps follow the accumulator tile by tile and signal the last one on
+    // last_full, a barrier that completes once: a parity wait on tfull from
+    // here could pass on an earlier phase of it.
     const int n_mine = blockIdx.x < ntiles ? (ntiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
     if (ok && n_mine > 0) {
-      if (!tc_wait(&tfull[0], unsigned(n_mine - 1) & 1u)) {
+      if (!tc_wait(last_full, 0u)) {
         ok = false;
       } else {
         tc_fence_after();
@@ -531,6 +536,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       if (!tc_wait(&tfull[0], unsigned(i) & 1u)) { ok = false; break; }
       tc_fence_after();
       const bool last = tile + int(gridDim.x) >= ntiles;
+      if (last && warp == kTcEpiWarp0 && lane == 0) tc_arrive(last_full);   // the unpack warps may join
       if (last)   // shared with the unpack warps: every fifth chunk of this quarter
         tc_drain(p, tmem, tile, row_tiles, quarter, lane, (warp - 2) >> 2, kTcLastDrainWarps / 4);
       else

@@ -792,6 +792,33 @@ def test_gemm_several_tiles_per_cta():
     assert mb.read_device_errors() == 0
 
 
+@pytest.mark.parametrize("precision", ["auto", "bf16"])
+def test_gemm_many_short_tiles_per_cta(precision):
+    # N = 128 is two 64-column stages per tile, fewer than the copy ring's
+    # slots, and 4096 rows x 8192 tokens make 16 x 32 tiles, so persistent CTAs
+    # take three or four tiles each: the last one is drained by all 20 warps
+    # only once it is in the accumulator.  Every output checked, for the split
+    # (mbok_gemm's choice at N = 128) and for the single bf16 tile.
+    import boolean_weight_matmul_b200 as mb
+    K, M, N, T = 2, 4096, 128, 8192
+    s = wl.random_signs(K, M, N, 891)
+    a = wl.alpha_decaying(K, M, N, 892)
+    X = wl.x_normal(T, N, 893)
+    prec = None if precision == "auto" else mb.GEMM_BF16
+    Y = gemm_gpu(packed_from_signs_gpu(s), alpha_blocked_gpu(a, K, M, N), K, M, N, X, precision=prec)
+    Y_ref, E = O.linear(O.pack_signs(s), a, K, M, N, X, "bf16")
+    if precision == "auto":
+        assert_close(Y, Y_ref, E, None, "gemm many short tiles", out_rel=BF16_OUT_REL)
+    else:
+        # A single bf16 tile: each weight rounded once (|dW| <= 2^-9 |W|, so
+        # |dy| <= 2^-9 sum|W x| = 2^-9 E) plus the output's own rounding,
+        # each bound taken with a factor 2 of margin, per element.
+        assert np.isfinite(Y).all()
+        bad = np.abs(Y - Y_ref) > 2.0 ** -8 * E + 2.0 ** -8 * np.abs(Y_ref) + 1e-6
+        assert not bad.any(), f"{int(bad.sum())} outputs outside the bf16-tile bound"
+    assert mb.read_device_errors() == 0
+
+
 def test_gemm_no_wait_gave_up():
     import boolean_weight_matmul_b200 as mb
     s = wl.random_signs(2, 256, 512, 991)
