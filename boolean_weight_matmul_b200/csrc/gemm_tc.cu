@@ -465,6 +465,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
         if (!ok) break;
         tc_commit(&tfull[0]);
+        if (tile + int(gridDim.x) >= ntiles) tc_commit(last_full);   // the unpack warps may join its drain
       }
     }
   } else if (warp < kTcEpiWarp0) {
@@ -514,10 +515,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         }
       }
     }
-    // The CTA's last tile: help the epilogue warps drain it.  The epilogue
-    // warps follow the accumulator tile by tile and signal the last one on
-    // last_full, a barrier that completes once: a parity wait on tfull from
-    // here could pass on an earlier phase of it.
+    // The CTA's last tile: help the epilogue warps drain it.  The MMA thread
+    // commits that tile to last_full as well as to tfull; last_full completes
+    // once, whereas a parity wait on tfull from here could pass on an earlier
+    // phase of it.
     const int n_mine = blockIdx.x < ntiles ? (ntiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
     if (ok && n_mine > 0) {
       if (!tc_wait(last_full, 0u)) {
@@ -536,7 +537,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       if (!tc_wait(&tfull[0], unsigned(i) & 1u)) { ok = false; break; }
       tc_fence_after();
       const bool last = tile + int(gridDim.x) >= ntiles;
-      if (last && warp == kTcEpiWarp0 && lane == 0) tc_arrive(last_full);   // the unpack warps may join
       if (last)   // shared with the unpack warps: every fifth chunk of this quarter
         tc_drain(p, tmem, tile, row_tiles, quarter, lane, (warp - 2) >> 2, kTcLastDrainWarps / 4);
       else
@@ -565,6 +565,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       (void)tc_wait(&tfull[b], 0u, kTcDrainNs);
       (void)tc_wait(&tfull[b], 1u, kTcDrainNs);
     }
+    (void)tc_wait(last_full, 0u, kTcDrainNs);
   }
   __syncthreads();
   if (warp == 1) {
