@@ -54,7 +54,7 @@ def args_parse():
                    help="profiling helper: run four launches of one GEMV (KERNEL as mbok_gemv_set_kernel: "
                         "0 auto, 1 lookup, 2 tensor, 3 slab lookup, 4 whole-row lookup) with L2 flushed "
                         "between them, print nothing else, and exit")
-    p.add_argument("--phase-profile", default=None, metavar="K,M,N,LAYERS",
+    p.add_argument("--phase-profile", default=None, metavar="K,M,N,LAYERS[,svid]",
                    help="per-phase split of the decode GEMV chain (profiling build with phase stamps)")
     p.add_argument("--profile-gemm", default=None, metavar="K,M,N,T,PRECISION",
                    help="profiling helper: run three launches of one prefill GEMM (PRECISION as "
@@ -766,7 +766,8 @@ def phase_profile(spec: str):
       drain       = last warp's copies drained - last warp out of the loop
       handoff_mid = first combine CTA past its wait - main kernel done
       combine     = last combine CTA done - first combine CTA past its wait
-    (the six terms add up to the layer's period)."""
+    (the six terms add up to the layer's period).  With a fifth field `svid` the
+    chain runs the rank-1 form (mbok_gemv_svid: one CTA per kernel and slab)."""
     import ctypes
     import statistics
     import torch
@@ -779,20 +780,38 @@ def phase_profile(spec: str):
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     S.mbok_gemv.argtypes = [vp, vp, i, i, i, i, vp, i, i, vp, vp, sz, vp]
     S.mbok_gemv.restype = i
+    S.mbok_gemv_svid.argtypes = [vp, vp, vp, i, i, i, vp, i, i, vp, vp, sz, vp]
+    S.mbok_gemv_svid.restype = i
     S.mbok_debug_phase_stamps.argtypes = [vp, sz, vp, sz]
     S.mbok_debug_phase_reset.argtypes = [i]
-    K, M, N, L = (int(v) for v in spec.split(","))
+    fields = spec.split(",")
+    svid = len(fields) == 5 and fields[4] == "svid"
+    assert len(fields) == 4 or svid, "K,M,N,LAYERS[,svid]"
+    K, M, N, L = (int(v) for v in fields[:4])
     assert 2 <= L <= 64
     dev = torch.device("cuda:0")
     packed, alphas, xs = build_layers(torch, mb, wl, K, M, N, L, dev, 4242)
     y = torch.empty(1, M, dtype=torch.float32, device=dev)
-    ws = mb.zeros_workspace(K, M, N, 1, dev)
+    if svid:
+        g = torch.Generator(device=dev)
+        g.manual_seed(4243)
+        s_in = [((torch.rand(K, N, device=dev, generator=g) * 0.4) + 0.8).to(torch.float16) for _ in range(L)]
+        s_out = [((torch.rand(K, M, device=dev, generator=g) * 0.4) + 0.8).mul(0.016).to(torch.float16)
+                 for _ in range(L)]
+        ws = mb.zeros_svid_workspace(K, M, N, 1, dev)
+    else:
+        ws = mb.zeros_workspace(K, M, N, 1, dev)
     stream = torch.cuda.Stream(device=dev)
 
     def chain():
         for l in range(L):
-            st = S.mbok_gemv(packed[l].data_ptr(), alphas[l].data_ptr(), K, M, N, 128, xs[l].data_ptr(),
-                             mb.BF16, 1, y.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            if svid:
+                st = S.mbok_gemv_svid(packed[l].data_ptr(), s_in[l].data_ptr(), s_out[l].data_ptr(), K, M, N,
+                                      xs[l].data_ptr(), mb.BF16, 1, y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                      stream.cuda_stream)
+            else:
+                st = S.mbok_gemv(packed[l].data_ptr(), alphas[l].data_ptr(), K, M, N, 128, xs[l].data_ptr(),
+                                 mb.BF16, 1, y.data_ptr(), ws.data_ptr(), ws.numel(), stream.cuda_stream)
             assert st == 0, st
 
     with torch.cuda.stream(stream):
@@ -847,7 +866,7 @@ def phase_profile(spec: str):
         for k, x in d.items():
             spread[k].append(x / 1000.0)
     med = {k: statistics.median(x) for k, x in terms.items()}
-    out = {"phase_profile": f"K={K} {M}x{N} batch 1, {L} layers, graph replay",
+    out = {"phase_profile": f"K={K} {M}x{N} batch 1, {L} layers, graph replay" + (", rank-1 form" if svid else ""),
            "main_ctas": nm, "combine_ctas": nc, "layer_us_events": round(per_layer_us, 3),
            "median_us": {k: round(x, 3) for k, x in med.items()},
            "share_of_period": {k: round(med[k] / med["period"], 3) for k in med if k != "period"},

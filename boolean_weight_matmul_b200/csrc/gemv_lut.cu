@@ -105,6 +105,8 @@ struct GemvParams {
   int weights_static;  // bits and scales may be read before the grid dependency wait
   int stamp_slot;      // profiling build only: this launch's phase-stamp slot
   int prefetch_octets; // octets per warp prefetched into L2 before the dependency wait
+  int sv_scales_staged; // rank-1 form: each octet's 8 output scales are copied with its bits
+                        // (M % 8 == 0 and s_out 16-byte aligned), not loaded after its lookups
 };
 
 // ---------------------------------------------------------------------------
@@ -225,6 +227,9 @@ __device__ __forceinline__ void issue_octet(const GemvParams& p, int slab, int u
   }
   if (!SV && lane < groups * K)
     cp_async16(st + G::kBits + lane * 16, p.alpha + alpha_offset(p.s, o, slab * kGroupsPerSlab, 0) + lane * 8);
+  // rank-1 form: rows 8o .. 8o+7 of s_out^kb into the stage's scale slot
+  if (SV && p.sv_scales_staged && lane == 0)
+    cp_async16(st + G::kBits, p.s_out + size_t(kb) * p.s.M + size_t(o) * kOctet);
   cp_async_commit();
 }
 
@@ -343,6 +348,10 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
         octet_dot<K>(tab, lane4, bits, al, acc);
       }
     }
+    // rank-1 form: this lane's row scale, read before the slot is refilled
+    float so = 0.f;
+    if (SV && p.sv_scales_staged)
+      so = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(st + G::kBits)[(lane >> 2) & 7]));
     __syncwarp();                  // all lanes are done reading the slot
     if (t + kDepth < n_mine)
       issue_octet<K, SV>(p, slab, units, groups, first + (t + kDepth) * kGemvWarps, kk, st, lane);
@@ -352,7 +361,14 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
     const int o = first + t * kGemvWarps;
     const int row = o * kOctet + ((lane >> 2) & 7);
     if ((lane & 3) == 0) {
-      if (SV) total = row < p.s.M ? total * __half2float(__ushort_as_half(p.s_out[size_t(kk) * p.s.M + row])) : 0.f;
+      if (SV) {
+        // A scale loaded here would hold the warp for a memory round trip
+        // per octet: the rank-1 loop took 5.25 us on q_proj (K = 3, 4096 x
+        // 4096) against 1.70 us for the grouped form's.
+        if (!p.sv_scales_staged && row < p.s.M)
+          so = __half2float(__ushort_as_half(p.s_out[size_t(kk) * p.s.M + row]));
+        total = row < p.s.M ? total * so : 0.f;
+      }
       if (nvs == 1) {
         if (row < p.s.M) p.y[row] = total;
       } else {
@@ -566,8 +582,8 @@ inline bool stage_early(bool weights_static, size_t packed_bytes) {
 inline int prefetch_depth(size_t packed_bytes) { return packed_bytes <= kEarlyStageMaxBytes ? kPrefetchOctets : 0; }
 
 static GemvParams make_params(const uint8_t* packed, const Shape& s, const void* x, float* y, void* workspace,
-                              bool weights_static, int nk) {
-  const GemvPlan pl = gemv_plan(s, device_sm_count(), nk);
+                              bool weights_static, int nk, int ctas_per_sm = 1) {
+  const GemvPlan pl = gemv_plan(s, device_sm_count() * ctas_per_sm, nk);
   GemvParams p;
   p.packed = packed;
   p.alpha = nullptr;
@@ -582,6 +598,7 @@ static GemvParams make_params(const uint8_t* packed, const Shape& s, const void*
   p.weights_static = stage_early(weights_static, size_t(s.O) * kOctet * s.K * (s.N / 8)) ? 1 : 0;
   p.stamp_slot = 0;
   p.prefetch_octets = prefetch_depth(size_t(s.O) * kOctet * s.K * (s.N / 8));
+  p.sv_scales_staged = 0;
   p.partial = pl.nslab * nk > 1 ? static_cast<float*>(workspace) : nullptr;
   return p;
 }
@@ -657,6 +674,7 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
     p.weights_static = early ? 1 : 0;
     p.stamp_slot = 0;
     p.prefetch_octets = prefetch_depth(launch_bytes);
+    p.sv_scales_staged = 0;
     p.partial = nslab > 1 ? static_cast<float*>(workspace) + poff : nullptr;
     mp.cta0[i] = cta;
     cm.partial[i] = p.partial;
@@ -704,14 +722,35 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
   return cudaGetLastError();
 }
 
+// CTAs of the rank-1 kernel that one SM holds at once (queried once per
+// device).  Its one-kernel stages leave room for two 512-thread CTAs per SM,
+// and its row ranges are sized for all of them.
+template <bool XF32>
+static int svid_ctas_per_sm() {
+  static PerDeviceValue<int> cache;
+  const int n = cache.get(current_device(), []() -> int {
+    const void* fn = reinterpret_cast<const void*>(gemv_lut8_kernel<1, XF32, true>);
+    int v = 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, StageGeom<1>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, kGemvThreads, StageGeom<1>::kSmem) != cudaSuccess)
+      return 0;
+    return v;
+  });
+  return n >= 1 ? n : 1;
+}
+
 // Rank-1 form: y = sum_k s_out^k (.) (B_k (s_in^k (.) x)) for one vector;
 // workspace as sized by gemv_svid_workspace_bytes.
 cudaError_t launch_gemv_svid(const uint8_t* packed, const uint16_t* s_in, const uint16_t* s_out, const Shape& s,
                              const void* x, bool x_f32, float* y, void* workspace, cudaStream_t stream,
                              bool weights_static) {
-  GemvParams p = make_params(packed, s, x, y, workspace, weights_static, s.K);
+  const int per_sm = x_f32 ? svid_ctas_per_sm<true>() : svid_ctas_per_sm<false>();
+  GemvParams p = make_params(packed, s, x, y, workspace, weights_static, s.K, per_sm);
   p.s_in = s_in;
   p.s_out = s_out;
+  // each octet's scales are one aligned 16-byte copy when M % 8 == 0
+  p.sv_scales_staged = (s.M % kOctet == 0 && (reinterpret_cast<uintptr_t>(s_out) & 15) == 0) ? 1 : 0;
   const int grid = p.nslab * p.nk * p.cps;
   return x_f32 ? launch_k<1, true, true>(p, grid, stream) : launch_k<1, false, true>(p, grid, stream);
 }

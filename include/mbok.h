@@ -226,7 +226,9 @@ size_t mbok_gemv_svid_workspace_bytes(int K, int M, int N, int batch);
  *     y[b][r] = sum_k s_out[k][r] * sum_j b_{k,r,j} * s_in[k][j] * x[b][j].
  *   packed : the K sign matrices in layout 1 (as for mbok_gemv).
  *   s_in   : fp16 [K][N] input scales, 16-byte aligned.
- *   s_out  : fp16 [K][M] output scales.
+ *   s_out  : fp16 [K][M] output scales; any 2-byte alignment.  With M a
+ *            multiple of 8 and s_out 16-byte aligned, each 8-row octet's
+ *            scales are copied into shared memory with its bits (faster).
  *   x, x_dtype, batch, y, workspace, workspace_bytes, stream: as mbok_gemv
  *            (workspace sized by mbok_gemv_svid_workspace_bytes).
  * Each product s_in * x is formed in fp32 (exact for bf16 x), the +-1 sums

@@ -494,7 +494,7 @@ def test_gemv_fused_projections_equal_separate_calls():
 # Rank-1 (SVID) scaled kernels
 # --------------------------------------------------------------------------
 
-def _svid_gpu(signs, s_in, s_out, x, x_dtype):
+def _svid_gpu(signs, s_in, s_out, x, x_dtype, s_out_offset=0):
     import torch
     import boolean_weight_matmul_b200 as mb
     K, M, N = signs.shape
@@ -502,6 +502,11 @@ def _svid_gpu(signs, s_in, s_out, x, x_dtype):
     packed = packed_from_signs_gpu(signs) if signs.dtype == np.int8 else signs
     si = to_dev(np.ascontiguousarray(s_in, dtype=np.float16).view(np.int16)).view(torch.float16)
     so = to_dev(np.ascontiguousarray(s_out, dtype=np.float16).view(np.int16)).view(torch.float16)
+    if s_out_offset:
+        # the same scales at an element offset inside a larger buffer
+        buf = torch.zeros(so.numel() + s_out_offset, dtype=torch.float16, device=so.device)
+        buf[s_out_offset:].copy_(so.reshape(-1))
+        so = buf[s_out_offset:].view(K, M)
     xd = x_dev(x, x_dtype)
     y = guarded((batch, M), torch.float32)
     ws = mb.zeros_svid_workspace(K, M, N, batch)
@@ -520,6 +525,19 @@ def test_gemv_svid_small_shapes(K, M, N, batch):
         y = _svid_gpu(s, s_in, s_out, x, x_dtype)
         y_ref, E = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, x_dtype)
         assert_close(y, y_ref, E, GEMV_REL_L2, f"svid K={K} M={M} N={N} b={batch} {x_dtype}")
+
+
+@pytest.mark.parametrize("K,M,N,offset", [(3, 64, 1536, 1), (2, 256, 4096, 4), (4, 136, 1024, 8)])
+def test_gemv_svid_output_scale_alignment(K, M, N, offset):
+    """s_out at a 2-, 8- or 16-byte offset with M % 8 == 0: the kernel copies
+    each octet's scales with its bits only from a 16-byte-aligned s_out, and
+    loads them one by one otherwise; both give the oracle's result."""
+    s = wl.random_signs(K, M, N, 8300 + K + M)
+    s_in, s_out = wl.svid_scales(K, M, N, 8301 + K + M)
+    x = wl.x_normal(2, N, 8302 + K + M)
+    y = _svid_gpu(s, s_in, s_out, x, "bf16", s_out_offset=offset)
+    y_ref, E = O.linear_svid(O.pack_signs(s), s_in, s_out, K, M, N, x, "bf16")
+    assert_close(y, y_ref, E, GEMV_REL_L2, f"svid K={K} M={M} N={N} s_out offset {offset}")
 
 
 @pytest.mark.parametrize("K,M,N,sample", [(3, 4096, 4096, None), (4, 13824, 5120, 256), (2, 4096, 11008, 256)])
