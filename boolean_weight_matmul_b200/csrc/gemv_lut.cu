@@ -727,15 +727,15 @@ cudaError_t launch_gemv_lut_multi(int nseg, const uint8_t* const* packed, const 
 // and its row ranges are sized for all of them.
 template <bool XF32>
 static int svid_ctas_per_sm() {
+  const void* fn = reinterpret_cast<const void*>(gemv_lut8_kernel<1, XF32, true>);
+  static PerDeviceOnce attr_once;   // the occupancy depends on the shared-memory attributes
+  if (set_smem_attr_once(attr_once, fn, StageGeom<1>::kSmem, true) != cudaSuccess) return 1;
   static PerDeviceValue<int> cache;
-  const int n = cache.get(current_device(), []() -> int {
-    const void* fn = reinterpret_cast<const void*>(gemv_lut8_kernel<1, XF32, true>);
+  const int n = cache.get(current_device(), [fn]() -> int {
     int v = 0;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, StageGeom<1>::kSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, kGemvThreads, StageGeom<1>::kSmem) != cudaSuccess)
-      return 0;
-    return v;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, kGemvThreads, StageGeom<1>::kSmem) == cudaSuccess
+               ? v
+               : 0;
   });
   return n >= 1 ? n : 1;
 }
