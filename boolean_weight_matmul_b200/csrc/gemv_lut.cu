@@ -301,6 +301,10 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
     prefetch_l2(static_cast<const unsigned char*>(p.x) + size_t(q) * kUnit * (XF32 ? 4 : 2));
     if (SV) prefetch_l2(p.s_in + size_t(kk) * p.s.N + size_t(q) * kUnit);
   }
+  // rank-1 form: the kernel's input scales for this lane's 8 columns -- a
+  // weight, so read before the wait when weights are static
+  uint4 sv = make_uint4(0u, 0u, 0u, 0u);
+  if (SV && lane_ok && p.weights_static) sv = *reinterpret_cast<const uint4*>(p.s_in + size_t(kk) * p.s.N + col0);
   allow_dependents();
   // x, the workspace and (unless static) the weights may be written by the
   // previous grid: wait for it.
@@ -312,7 +316,7 @@ __device__ __forceinline__ void gemv_lut8_body(const GemvParams& p, int bid) {
   load_x8<XF32>(p.x, col0, lane_ok, xv);
   if (SV && lane_ok) {
     // rank-1 form: the kernel's input scale, applied before the tables
-    const uint4 sv = *reinterpret_cast<const uint4*>(p.s_in + size_t(kk) * p.s.N + col0);
+    if (!p.weights_static) sv = *reinterpret_cast<const uint4*>(p.s_in + size_t(kk) * p.s.N + col0);
     const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
