@@ -283,8 +283,9 @@ int mbok_gemv_multi(int nseg, const uint32_t* const* packed, const uint16_t* con
  * Returns MBOK_ERR_INVALID_ARG for any other value. */
 int mbok_gemv_set_kernel(int kernel);
 
-/* Whether the GEMV kernels may read their weights (packed bits and scales)
- * before waiting for the preceding launch in the stream.  GEMV launches use
+/* Whether the GEMV kernels may read their weights (packed bits and scales:
+ * alpha, or s_in and s_out for mbok_gemv_svid) before waiting for the
+ * preceding launch in the stream.  GEMV launches use
  * programmatic dependent launch: a GEMV may start while the kernel before it
  * finishes, if that kernel signalled early (griddepcontrol.launch_dependents);
  * everything it reads after its wait is ordered after that kernel.  With
