@@ -254,6 +254,13 @@ def build_layers(torch, mb, wl, K, M, N, L, dev, seed0):
     return packed, alphas, xs
 
 
+def e2e_copy_cuts(L: int):
+    """Layer boundaries of the pipelined end-to-end step's host copies: inputs
+    [0, 4) then [4, L); outputs [0, L - 4) then [L - 4, L).  Copy i covers
+    layers cuts[i] .. cuts[i+1] - 1."""
+    return sorted({0, min(4, L), L}), sorted({0, max(L - 4, 0), L})
+
+
 def time_graph(torch, fn, steps, warmup, stream):
     """Capture fn() once, replay warmup + steps times; returns ms per replay."""
     with torch.cuda.stream(stream):
@@ -396,8 +403,7 @@ def run_gpu(a):
     # the overlap of their launches (5 chunks each way measured 258 us per
     # step, a third output copy at the halfway layer 248 us, this 246 us).
     cs = torch.cuda.Stream(device=dev)
-    in_cuts = sorted({0, min(4, L), L})
-    out_cuts = sorted({0, max(L - 4, 0), L})
+    in_cuts, out_cuts = e2e_copy_cuts(L)
     chunks = len(in_cuts) - 1 + len(out_cuts) - 1
 
     def e2e_step_pipelined():
