@@ -56,6 +56,9 @@ def args_parse():
                         "between them, print nothing else, and exit")
     p.add_argument("--phase-profile", default=None, metavar="K,M,N,LAYERS[,svid]",
                    help="per-phase split of the decode GEMV chain (profiling build with phase stamps)")
+    p.add_argument("--profile-convert", default=None, metavar="K,M,N",
+                   help="profiling helper: run two launches each of residual binarisation (fp32 W) and bit "
+                        "packing (int8 signs) with L2 flushed before each, print nothing else, and exit")
     p.add_argument("--profile-gemm", default=None, metavar="K,M,N,T,PRECISION",
                    help="profiling helper: run three launches of one prefill GEMM (PRECISION as "
                         "mbok_gemm_ex: 0 auto, 1 bf16, 2 split), print nothing else, and exit")
@@ -788,6 +791,31 @@ def profile_gemv(spec: str):
     torch.cuda.synchronize()
 
 
+def profile_convert(spec: str):
+    """Two launches each of residual binarisation and bit packing on random
+    inputs, with L2 flushed before each launch (for an ncu capture)."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    mbuild.build()
+    K, M, N = (int(v) for v in spec.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    W = torch.randn(M, N, device=dev, generator=g) * 0.02
+    R = torch.empty_like(W)
+    S = torch.randint(-1, 1, (K, M, N), dtype=torch.int8, device=dev, generator=g)
+    packed = mb.empty_packed(K, M, N, dev)
+    alpha = mb.empty_alpha(K, M, N, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2
+    for _ in range(2):
+        flush.zero_()
+        mb.residual_binarize(W, M, N, K, 128, packed, alpha, R)
+        flush.zero_()
+        mb.pack_bits(S, K, M, N, packed)
+    torch.cuda.synchronize()
+
+
 def profile_gemm(spec: str):
     """Three launches of one prefill GEMM on random weights (for an ncu capture)."""
     import torch
@@ -938,6 +966,9 @@ def main():
         return
     if a.profile_gemm:
         profile_gemm(a.profile_gemm)
+        return
+    if a.profile_convert:
+        profile_convert(a.profile_convert)
         return
     if a.impl == "reference":
         run_reference(a)
