@@ -56,6 +56,9 @@ def args_parse():
                         "between them, print nothing else, and exit")
     p.add_argument("--phase-profile", default=None, metavar="K,M,N,LAYERS[,svid]",
                    help="per-phase split of the decode GEMV chain (profiling build with phase stamps)")
+    p.add_argument("--profile-svid", default=None, metavar="K,M,N",
+                   help="profiling helper: run four launches of the rank-1-form GEMV (batch 1) with L2 flushed "
+                        "between them, print nothing else, and exit")
     p.add_argument("--profile-convert", default=None, metavar="K,M,N",
                    help="profiling helper: run two launches each of residual binarisation (fp32 W) and bit "
                         "packing (int8 signs) with L2 flushed before each, print nothing else, and exit")
@@ -791,6 +794,31 @@ def profile_gemv(spec: str):
     torch.cuda.synchronize()
 
 
+def profile_svid(spec: str):
+    """Four launches of the rank-1-form GEMV on random weights and scales, with
+    L2 flushed before each (for an ncu capture)."""
+    import torch
+    import boolean_weight_matmul_b200 as mb
+    from boolean_weight_matmul_b200 import build as mbuild
+    mbuild.build()
+    K, M, N = (int(v) for v in spec.split(","))
+    dev = torch.device("cuda:0")
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (mb.packed_bytes(K, M, N) // 4,), dtype=torch.int32,
+                           device=dev, generator=g)
+    s_in = ((torch.rand(K, N, device=dev, generator=g) * 0.4) + 0.8).to(torch.float16)
+    s_out = ((torch.rand(K, M, device=dev, generator=g) * 0.4) + 0.8).mul(0.016).to(torch.float16)
+    x = torch.randn(1, N, device=dev, generator=g).to(torch.bfloat16)
+    y = torch.empty(1, M, dtype=torch.float32, device=dev)
+    ws = mb.zeros_svid_workspace(K, M, N, 1, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2
+    for _ in range(4):
+        flush.zero_()
+        mb.gemv_svid(packed, s_in, s_out, K, M, N, x, mb.BF16, 1, y, ws)
+    torch.cuda.synchronize()
+
+
 def profile_convert(spec: str):
     """Two launches each of residual binarisation and bit packing on random
     inputs, with L2 flushed before each launch (for an ncu capture)."""
@@ -969,6 +997,9 @@ def main():
         return
     if a.profile_convert:
         profile_convert(a.profile_convert)
+        return
+    if a.profile_svid:
+        profile_svid(a.profile_svid)
         return
     if a.impl == "reference":
         run_reference(a)
