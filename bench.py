@@ -61,7 +61,8 @@ def args_parse():
                         "between them, print nothing else, and exit")
     p.add_argument("--profile-convert", default=None, metavar="K,M,N",
                    help="profiling helper: run two launches each of residual binarisation (fp32 W) and bit "
-                        "packing (int8 signs) with L2 flushed before each, print nothing else, and exit")
+                        "packing (int8 signs), then one scale refit and one successive-SVID conversion, "
+                        "with L2 flushed before each, print nothing else, and exit")
     p.add_argument("--profile-gemm", default=None, metavar="K,M,N,T,PRECISION",
                    help="profiling helper: run three launches of one prefill GEMM (PRECISION as "
                         "mbok_gemm_ex: 0 auto, 1 bf16, 2 split), print nothing else, and exit")
@@ -821,7 +822,8 @@ def profile_svid(spec: str):
 
 def profile_convert(spec: str):
     """Two launches each of residual binarisation and bit packing on random
-    inputs, with L2 flushed before each launch (for an ncu capture)."""
+    inputs, then one scale refit and one successive-SVID conversion, with L2
+    flushed before each call (for an ncu capture)."""
     import torch
     import boolean_weight_matmul_b200 as mb
     from boolean_weight_matmul_b200 import build as mbuild
@@ -841,6 +843,15 @@ def profile_convert(spec: str):
         mb.residual_binarize(W, M, N, K, 128, packed, alpha, R)
         flush.zero_()
         mb.pack_bits(S, K, M, N, packed)
+    flush.zero_()
+    mb.residual_binarize(W, M, N, K, 128, packed, alpha, R)
+    flush.zero_()
+    mb.refit_alpha(W, packed, K, M, N, 128, alpha)
+    s_in = torch.empty(K, N, dtype=torch.float16, device=dev)
+    s_out = torch.empty(K, M, dtype=torch.float16, device=dev)
+    svws = torch.empty(int(mb.lib().mbok_svid_workspace_bytes(M, N)), dtype=torch.uint8, device=dev)
+    flush.zero_()
+    mb.svid_binarize(W, M, N, K, 6, packed, s_in, s_out, R, svws)
     torch.cuda.synchronize()
 
 

@@ -137,21 +137,43 @@ __global__ void __launch_bounds__(kSvThreads) svid_sign_update_kernel(float* __r
   float sin_f[kUnit];
 #pragma unroll
   for (int b = 0; b < kUnit; ++b) sin_f[b] = __half2float(s_in[q * kUnit + b]);
+  // The unit's 16 residuals of a row are 64 contiguous bytes (16-byte aligned:
+  // R is, and N is a multiple of 128): four 16-byte loads and stores, for four
+  // rows at a time, instead of 16 scalar accesses per row (the same
+  // arithmetic per element).  The scalar form ran at 1.0 TB/s (355 us per
+  // kernel at 11008 x 4096); this one took the whole K = 3 conversion from
+  // 2.49 to 1.60 ms.
   uint32_t h[kOctet];
 #pragma unroll
-  for (int i = 0; i < kOctet; ++i) {
-    const int r = o * kOctet + i;
-    h[i] = 0;
-    if (r >= s.M) continue;
-    const float so = __half2float(s_out[r]);
-    float* row = R + size_t(r) * s.N + size_t(q) * kUnit;
+  for (int i0 = 0; i0 < kOctet; i0 += 4) {
+    float4 v[4][4];
 #pragma unroll
-    for (int b = 0; b < kUnit; ++b) {
-      const float x = row[b];
-      const bool pos = x >= 0.f;
-      h[i] |= uint32_t(pos) << b;
-      const float p = __fmul_rn(so, sin_f[b]);
-      row[b] = __fsub_rn(x, pos ? p : -p);
+    for (int i = 0; i < 4; ++i) {
+      const int r = o * kOctet + i0 + i;
+      const float4* src = reinterpret_cast<const float4*>(R + size_t(r) * s.N + size_t(q) * kUnit);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[i][c] = r < s.M ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = o * kOctet + i0 + i;
+      h[i0 + i] = 0;
+      if (r >= s.M) continue;
+      const float so = __half2float(s_out[r]);
+      float4* dst = reinterpret_cast<float4*>(R + size_t(r) * s.N + size_t(q) * kUnit);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float e[4] = {v[i][c].x, v[i][c].y, v[i][c].z, v[i][c].w};
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+          const int b = 4 * c + d;
+          const bool pos = e[d] >= 0.f;
+          h[i0 + i] |= uint32_t(pos) << b;
+          const float p = __fmul_rn(so, sin_f[b]);
+          e[d] = __fsub_rn(e[d], pos ? p : -p);
+        }
+        dst[c] = make_float4(e[0], e[1], e[2], e[3]);
+      }
     }
   }
   uint4 out;
